@@ -1,0 +1,226 @@
+/*
+ * wf_attn.h -- C ABI of the B200 (sm_100a) attention-forward library.
+ *
+ * One operation, the scaled-dot-product attention forward
+ *
+ *     out = softmax(Q * K^T * qkScale + mask) * V
+ *
+ * with GQA head grouping, boolean keep-masks, additive float masks, in-kernel
+ * causal masks, packed variable-length sequences and the MLA split
+ * contraction q*k + qRope*kRope; plus the rolling sink+window BlockKVCache
+ * that feeds it.
+ *
+ * Sources the calls follow:
+ *   [P1]  "Core 注意力", WorldFoundry docs (openenvision.github.io/WorldFoundry),
+ *         sections "选择最窄的入口" (SDPA contract, GQA expansion),
+ *         "一个可以在 CPU 或 GPU 上运行的例子" (layouts [B,H,L,D], bool mask =
+ *         keep, float mask added) and "Block KV cache 的调用顺序" (cache calls,
+ *         their order, sink and window sizes).
+ *   [P2]  "MLA Prefill", CANN ATB docs (hiascend.com), "定义" (a C interface
+ *         that returns a status) and the parameter table (Q/QRope/K/kRope/V,
+ *         qSeqLen/kvSeqLen, mask, headNum, qkScale, kvHeadNum, maskType,
+ *         attenOut).
+ *
+ * Conventions for every call:
+ *   - All tensor data pointers are DEVICE pointers of the current CUDA device
+ *     unless a parameter says "host".  The library never frees caller memory.
+ *   - Tensors are described by wf_tensor_t: dims and strides are in ELEMENTS;
+ *     the last dimension must have stride 1.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Launches are asynchronous on that stream.
+ *   - Argument errors are reported synchronously, before anything is
+ *     launched; wf_last_error_message() then holds a description.
+ *   - Device-side conditions that can only be seen while running (bad
+ *     sequence lengths, a bounded wait that ran out) are recorded in a device
+ *     status word read by wf_get_device_status().
+ *   - Not thread-safe per wf_kvcache_t handle; the attention call is
+ *     reentrant across host threads.
+ */
+#ifndef WF_ATTN_H
+#define WF_ATTN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define WF_ATTN_VERSION 1
+
+/* Status codes (the [P2] "定义" section returns a status from every call). */
+typedef enum wf_status {
+    WF_OK = 0,
+    WF_ERR_INVALID_ARG = 1,   /* shape / stride / dtype / pointer is not valid */
+    WF_ERR_UNSUPPORTED = 2,   /* valid request outside what the kernels implement */
+    WF_ERR_ORDER = 3,         /* BlockKVCache call out of the documented order */
+    WF_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
+    WF_ERR_NO_MEMORY = 5,     /* host or device allocation failed */
+    WF_ERR_TIMEOUT = 6,       /* a bounded device wait ran out (device status) */
+    WF_ERR_NO_DEVICE = 7      /* no usable sm_100 device for this call */
+} wf_status_t;
+
+/* Element types.  WF_U8 is the boolean keep-mask type (nonzero = keep). */
+typedef enum wf_dtype {
+    WF_F32 = 0,
+    WF_BF16 = 1,
+    WF_F16 = 2,   /* reserved: not accepted by wf_attn_fwd yet */
+    WF_U8 = 3,
+    WF_I32 = 4
+} wf_dtype_t;
+
+/* maskType.  [P2] table row "maskType" (UNDEFINED / SPEC / MASK_FREE) and row
+ * "Mask" (CAUSAL_MASK may pass nullptr); [P1] example section for the two
+ * explicit mask kinds.  ATB names map as: UNDEFINED -> NONE; CAUSAL_MASK,
+ * MASK_FREE, SPEC -> CAUSAL (generated in the kernel; no mask tensor read). */
+typedef enum wf_mask_type {
+    WF_MASK_NONE = 0,
+    WF_MASK_CAUSAL = 1,     /* key j visible to query i iff j <= i + (Lk - Lq) */
+    WF_MASK_BOOL_KEEP = 2,  /* mask dtype WF_U8, nonzero = keep               */
+    WF_MASK_ADDITIVE = 3    /* mask dtype = q dtype or WF_F32, added to scores */
+} wf_mask_type_t;
+
+/* Tensor descriptor: up to 4 dims, strides in elements, caller-owned data. */
+typedef struct wf_tensor {
+    void *data;
+    int32_t dtype;          /* wf_dtype_t */
+    int32_t ndim;
+    int64_t shape[4];
+    int64_t stride[4];
+} wf_tensor_t;
+
+/*
+ * wf_attn_fwd -- attention forward.  [P2] "定义" + parameter table (argument
+ * set; headNum/kvHeadNum/qkScale), [P1] "选择最窄的入口" (SDPA contract, GQA).
+ *
+ * Two layouts, chosen by whether qSeqLen is given:
+ *
+ *   dense  (qSeqLen == kvSeqLen == NULL), the [P1] example layout:
+ *     q   [B, headNum,   Lq, Dqk]     out [B, headNum, Lq, Dv]
+ *     k   [B, kvHeadNum, Lk, Dqk]     v   [B, kvHeadNum, Lk, Dv]
+ *   packed (qSeqLen, kvSeqLen given), the [P2] table layout:
+ *     q   [nTokens,   headNum,   Dqk]  out [nTokens, headNum, Dv]
+ *     k   [nKvTokens, kvHeadNum, Dqk]  v   [nKvTokens, kvHeadNum, Dv]
+ *     qSeqLen, kvSeqLen: WF_I32 [batch] DEVICE arrays; sequence b occupies
+ *     rows [sum_{c<b} len_c, sum_{c<=b} len_c).  The lengths are read on the
+ *     device; if they sum past nTokens / nKvTokens (or are negative) the
+ *     call computes nothing and the device status becomes
+ *     WF_ERR_INVALID_ARG.
+ *
+ *   qRope / kRope (MLA, [P2] rows QRope/kRope): NULL, or [.., headNum, 64] /
+ *     [.., kvHeadNum, 64] in the same layout as q / k.  Scores are then
+ *     qkScale * (q.k + qRope.kRope).  Both or neither.
+ *   mask: used only for WF_MASK_BOOL_KEEP / WF_MASK_ADDITIVE, dense layout
+ *     only: logical [B, headNum, Lq, Lk]; a stride of 0 broadcasts a dim
+ *     (size-1 dims must be given with stride 0 or size equal to the full
+ *     extent).  Must be NULL otherwise.
+ *   headNum % kvHeadNum == 0; query head h reads kv head h / (headNum/kvHeadNum).
+ *   qkScale multiplies Q*K^T before the mask is added ([P2] row qkScale).
+ *   dtypes: q, k, v, qRope, kRope, out all WF_BF16, or all WF_F32 (the F32
+ *     path multiplies on TF32 tensor cores).  Dqk, Dv in {64, 96, 128};
+ *     with rope: Dqk = 128, Dv = 128, BF16.
+ *   Alignment: every data pointer 16-byte aligned; every stride except the
+ *     last a multiple of 16 bytes.
+ *   A query row that sees no key (causal with Lq > Lk, or an all-false
+ *   keep-mask row) produces zeros.
+ *
+ * Returns WF_OK once launched (asynchronous), an argument status otherwise.
+ * Ownership: all tensors are the caller's.  The library keeps a per-device
+ * workspace (schedule tables) that it grows on demand and frees in
+ * wf_shutdown().
+ */
+wf_status_t wf_attn_fwd(const wf_tensor_t *q, const wf_tensor_t *qRope,
+                        const wf_tensor_t *k, const wf_tensor_t *kRope,
+                        const wf_tensor_t *v,
+                        const wf_tensor_t *qSeqLen, const wf_tensor_t *kvSeqLen,
+                        const wf_tensor_t *mask,
+                        int32_t headNum, int32_t kvHeadNum, float qkScale,
+                        int32_t maskType, wf_tensor_t *out, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * BlockKVCache ([P1] "Block KV cache 的调用顺序").
+ *
+ * The caller owns two buffers k_buf / v_buf of logical shape
+ * [B, H, L, Dk] / [B, H, L, Dv] (seq_dim = 2), or [B, L, H, D] (seq_dim = 1);
+ * L = sink_size + window_size, a multiple of chunk_size; sink_size is also a
+ * multiple of chunk_size and window_size >= chunk_size.  The handle only
+ * records the rolling state; the buffers are written by wf_kvcache_update.
+ *
+ * Every chunk index c runs  before_update(c) -> update -> cached -> after_update(c).
+ * before_update(c) is legal when no chunk is in progress and c == 0 (first
+ * chunk), c == last committed (overwrite the same logical chunk) or
+ * c == last committed + 1 (append, or roll the window).  Anything else returns
+ * WF_ERR_ORDER and leaves the state as it was.
+ *
+ * Chunk c lives in slot c while c < sink/chunk, afterwards in
+ * sink/chunk + (c - sink/chunk) mod (window/chunk); slot s covers sequence
+ * positions [s*chunk, (s+1)*chunk) of the buffers.  After chunk c the visible
+ * tokens are the physical prefix of chunk * min(c+1, L/chunk) positions.
+ * ------------------------------------------------------------------------- */
+typedef struct wf_kvcache wf_kvcache_t;
+
+/* Create a handle over caller-owned buffers (4-d, same dtype, last dim
+ * contiguous).  No device memory is touched.  *out receives the handle. */
+wf_status_t wf_kvcache_create(const wf_tensor_t *k_buf, const wf_tensor_t *v_buf,
+                              int32_t seq_dim, int64_t chunk_size,
+                              int64_t sink_size, int64_t window_size,
+                              wf_kvcache_t **out);
+
+/* Start chunk `chunk_idx` (host only, no device work). */
+wf_status_t wf_kvcache_before_update(wf_kvcache_t *cache, int64_t chunk_idx);
+
+/* Write the current chunk: k / v have the buffers' shape with exactly
+ * chunk_size positions along seq_dim; copied on `stream` into the chunk's
+ * slot. */
+wf_status_t wf_kvcache_update(wf_kvcache_t *cache, const wf_tensor_t *k,
+                              const wf_tensor_t *v, void *stream);
+
+/* Views of the visible prefix, returned in the logical [B, H, vis, D] form
+ * (strides of the buffers), ready to pass to wf_attn_fwd as k / v.  Physical
+ * ring order: attention without a causal mask does not depend on key order.
+ * Host only. */
+wf_status_t wf_kvcache_cached(wf_kvcache_t *cache, wf_tensor_t *k_view,
+                              wf_tensor_t *v_view, int64_t *visible_len);
+
+/* Commit chunk `chunk_idx` (must equal the one in progress). Host only. */
+wf_status_t wf_kvcache_after_update(wf_kvcache_t *cache, int64_t chunk_idx);
+
+/* Read the state: index in progress (-1 before the first), last committed
+ * index (-1 before the first commit), slot of the index in progress (-1 if
+ * none), visible length, phase (0 idle, 1 before_update done, 2 update done,
+ * 3 cached done).  Any output pointer may be NULL. */
+wf_status_t wf_kvcache_get_state(const wf_kvcache_t *cache, int64_t *cur_idx,
+                                 int64_t *committed_idx, int64_t *write_slot,
+                                 int64_t *visible_len, int32_t *phase);
+
+/* Copy the visible tokens in LOGICAL chunk order (sink chunks, then the
+ * window's chunks oldest first) into k_out / v_out, [B, H, vis, D] (or the
+ * seq_dim = 1 form).  Allowed in the same phases as wf_kvcache_cached. */
+wf_status_t wf_kvcache_gather_logical(wf_kvcache_t *cache, wf_tensor_t *k_out,
+                                      wf_tensor_t *v_out, void *stream);
+
+void wf_kvcache_destroy(wf_kvcache_t *cache);
+
+/* ---------------------------------------------------------------------------
+ * Diagnostics and lifetime.
+ * ------------------------------------------------------------------------- */
+
+/* Synchronize `stream`, then read and clear the current device's status
+ * word: WF_OK, WF_ERR_TIMEOUT (a bounded wait inside a kernel ran out; the
+ * kernel abandoned its work and the affected output is undefined) or
+ * WF_ERR_INVALID_ARG (device-side length check failed). */
+wf_status_t wf_get_device_status(void *stream);
+
+/* Description of the last error on the calling host thread ("" if none). */
+const char *wf_last_error_message(void);
+
+/* Library version (WF_ATTN_VERSION). */
+int32_t wf_version(void);
+
+/* Free the per-device workspaces.  Call with no work in flight. */
+void wf_shutdown(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WF_ATTN_H */

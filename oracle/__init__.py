@@ -1,0 +1,14 @@
+"""fp64 CPU oracle for the attention forward and the BlockKVCache.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package.  The CUDA library never
+calls it, and it never imports the CUDA library: the only thing the two sides
+share is the seeded input generator module, which holds none of the method's
+arithmetic.
+
+Contents:
+  * ``sdpa`` / ``sdpa_rows``  -- ctypes front end of ``sdpa_oracle.c`` (fp64, OpenMP)
+  * ``brute``                 -- pure-Python per-element loops for tiny inputs
+  * ``kvcache_model``         -- plain Python model of the BlockKVCache contract
+"""
+from .sdpa import sdpa, sdpa_rows, build_oracle, oracle_threads, MASK_KINDS  # noqa: F401
