@@ -1,0 +1,219 @@
+"""Python front end: torch tensors in, C-ABI calls out.
+
+Every function here only marshals arguments (pointers, shapes, strides, the
+current CUDA stream) into ``libwfattn.so``; all computation runs in its
+kernels.  Tensors must live on a CUDA device: there is no CPU path.
+
+Mirrors the pages' API surface:
+  * :func:`attn_fwd` -- the attention forward of "Core 注意力" (section
+    "选择最窄的入口", PyTorch SDPA contract with GQA) and of "MLA Prefill"
+    (packed layout, qSeqLen/kvSeqLen, QRope/kRope, headNum/kvHeadNum/qkScale).
+  * :class:`BlockKVCache` -- the rolling cache of "Core 注意力", section
+    "Block KV cache 的调用顺序" (before_update -> update -> cached_k/cached_v
+    -> after_update).
+"""
+from __future__ import annotations
+
+import ctypes
+import enum
+import math
+
+import torch
+
+from . import _lib as L
+
+
+class WfError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{L.STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+class MaskType(enum.IntEnum):
+    NONE = L.WF_MASK_NONE
+    CAUSAL = L.WF_MASK_CAUSAL
+    BOOL_KEEP = L.WF_MASK_BOOL_KEEP
+    ADDITIVE = L.WF_MASK_ADDITIVE
+
+
+_DTYPES = {torch.float32: L.WF_F32, torch.bfloat16: L.WF_BF16, torch.float16: L.WF_F16,
+           torch.uint8: L.WF_U8, torch.bool: L.WF_U8, torch.int32: L.WF_I32}
+
+
+def _check(status: int) -> None:
+    if status != L.WF_OK:
+        msg = L.load().wf_last_error_message()
+        raise WfError(status, msg.decode() if msg else "")
+
+
+def describe(t: torch.Tensor | None) -> L.WfTensor | None:
+    """C descriptor of a tensor (no copy; the tensor must outlive the call)."""
+    if t is None:
+        return None
+    if t.dim() > 4:
+        raise ValueError("at most 4 dims")
+    d = L.WfTensor()
+    d.data = t.data_ptr() if t.numel() else None
+    d.dtype = _DTYPES[t.dtype]
+    d.ndim = t.dim()
+    for i in range(t.dim()):
+        d.shape[i] = t.shape[i]
+        d.stride[i] = t.stride(i)
+    return d
+
+
+def _ref(d):
+    return ctypes.byref(d) if d is not None else None
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _require_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise WfError(L.WF_ERR_INVALID_ARG,
+                          "tensors must be on a CUDA device (this library has no CPU path)")
+
+
+def attn_fwd(q, k, v, *, qrope=None, krope=None, q_seqlen=None, kv_seqlen=None, mask=None,
+             mask_type=None, head_num=None, kv_head_num=None, qk_scale=None, out=None,
+             stream=None, debug_flags=0, timeout_cycles=0):
+    """out = softmax(q k^T * qk_scale + mask) v, see ``include/wf_attn.h``.
+
+    Dense: q [B,Hq,Lq,D], k/v [B,Hkv,Lk,D].  Packed: q [T,Hq,D], k/v [Tk,Hkv,D]
+    with int32 ``q_seqlen`` / ``kv_seqlen`` on the device.  ``mask_type``
+    defaults to BOOL_KEEP for a bool mask, ADDITIVE for a float mask, NONE
+    otherwise.  ``qk_scale`` defaults to 1/sqrt(Dqk + Drope).
+    """
+    _require_cuda(q, k, v, qrope, krope, q_seqlen, kv_seqlen, mask, out)
+    varlen = q_seqlen is not None
+    if head_num is None:
+        head_num = q.shape[1]
+    if kv_head_num is None:
+        kv_head_num = k.shape[1]
+    if mask_type is None:
+        if mask is None:
+            mask_type = MaskType.NONE
+        else:
+            mask_type = MaskType.BOOL_KEEP if mask.dtype in (torch.bool, torch.uint8) else MaskType.ADDITIVE
+    if qk_scale is None:
+        qk_scale = 1.0 / math.sqrt(q.shape[-1] + (qrope.shape[-1] if qrope is not None else 0))
+    if out is None:
+        shape = (q.shape[0], head_num, v.shape[-1]) if varlen else \
+            (q.shape[0], head_num, q.shape[2], v.shape[-1])
+        out = torch.empty(shape, dtype=q.dtype, device=q.device)
+    if mask is not None and mask.dtype == torch.bool:
+        mask = mask.view(torch.uint8)
+    if mask is not None:
+        while mask.dim() < 4:
+            mask = mask.unsqueeze(0)
+    descs = [describe(x) for x in (q, qrope, k, krope, v, q_seqlen, kv_seqlen, mask)]
+    od = describe(out)
+    lib = L.load()
+    with torch.cuda.device(q.device):
+        if debug_flags or timeout_cycles:
+            st = lib.wf_attn_fwd_debug(*[_ref(d) for d in descs], int(head_num), int(kv_head_num),
+                                       float(qk_scale), int(mask_type), ctypes.byref(od),
+                                       _stream(stream), int(debug_flags), int(timeout_cycles))
+        else:
+            st = lib.wf_attn_fwd(*[_ref(d) for d in descs], int(head_num), int(kv_head_num),
+                                 float(qk_scale), int(mask_type), ctypes.byref(od), _stream(stream))
+    _check(st)
+    return out
+
+
+def device_status(stream=None) -> None:
+    """Synchronize the stream and raise if a kernel recorded a device-side error."""
+    _check(L.load().wf_get_device_status(_stream(stream)))
+
+
+class BlockKVCache:
+    """Rolling sink + window KV cache over caller-owned buffers.
+
+    ``k_buf``/``v_buf``: [B, H, L, D] (seq_dim 2) or [B, L, H, D] (seq_dim 1) on a
+    CUDA device.  ``sink_size + window_size == L``; both multiples of
+    ``chunk_size``.  State transitions are checked by the library; a call out
+    of order raises :class:`WfError` with status ``WF_ERR_ORDER``.
+    """
+
+    def __init__(self, k_buf, v_buf, *, seq_dim=2, chunk_size, window_size, sink_size=0):
+        _require_cuda(k_buf, v_buf)
+        self.k_buf, self.v_buf = k_buf, v_buf
+        self.seq_dim = seq_dim
+        h = ctypes.c_void_p()
+        self._kd, self._vd = describe(k_buf), describe(v_buf)
+        _check(L.load().wf_kvcache_create(ctypes.byref(self._kd), ctypes.byref(self._vd), seq_dim,
+                                          chunk_size, sink_size, window_size, ctypes.byref(h)))
+        self._h = h
+
+    @classmethod
+    def allocate(cls, k_shape, v_shape, *, seq_dim=2, chunk_size, window_size, sink_size=0,
+                 device="cuda", dtype=torch.bfloat16):
+        """Allocate zeroed buffers of the given shapes and wrap them."""
+        kb = torch.zeros(k_shape, dtype=dtype, device=device)
+        vb = torch.zeros(v_shape, dtype=dtype, device=device)
+        return cls(kb, vb, seq_dim=seq_dim, chunk_size=chunk_size, window_size=window_size,
+                   sink_size=sink_size)
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h is not None and h.value:
+            L.load().wf_kvcache_destroy(h)
+            self._h = None
+
+    def before_update(self, chunk_idx: int) -> None:
+        _check(L.load().wf_kvcache_before_update(self._h, int(chunk_idx)))
+
+    def update(self, k, v, stream=None) -> None:
+        _require_cuda(k, v)
+        kd, vd = describe(k), describe(v)
+        with torch.cuda.device(self.k_buf.device):
+            _check(L.load().wf_kvcache_update(self._h, ctypes.byref(kd), ctypes.byref(vd),
+                                              _stream(stream)))
+
+    def _views(self):
+        kd, vd, vis = L.WfTensor(), L.WfTensor(), ctypes.c_int64()
+        _check(L.load().wf_kvcache_cached(self._h, ctypes.byref(kd), ctypes.byref(vd),
+                                          ctypes.byref(vis)))
+        kv = torch.as_strided(self.k_buf, tuple(kd.shape[:4]), tuple(kd.stride[:4]))
+        vv = torch.as_strided(self.v_buf, tuple(vd.shape[:4]), tuple(vd.stride[:4]))
+        return kv, vv
+
+    def cached_k(self):
+        """Visible keys, [B, H, vis, D] view of the buffer (physical ring order)."""
+        return self._views()[0]
+
+    def cached_v(self):
+        """Visible values, [B, H, vis, D] view of the buffer (physical ring order)."""
+        return self._views()[1]
+
+    def after_update(self, chunk_idx: int) -> None:
+        _check(L.load().wf_kvcache_after_update(self._h, int(chunk_idx)))
+
+    def state(self):
+        """(current index, committed index, write slot, visible length, phase)."""
+        cur, com, slot, vis = (ctypes.c_int64() for _ in range(4))
+        ph = ctypes.c_int32()
+        _check(L.load().wf_kvcache_get_state(self._h, ctypes.byref(cur), ctypes.byref(com),
+                                             ctypes.byref(slot), ctypes.byref(vis),
+                                             ctypes.byref(ph)))
+        return cur.value, com.value, slot.value, vis.value, ph.value
+
+    def gather_logical(self, stream=None):
+        """Copy of the visible tokens in logical chunk order (buffer layout)."""
+        vis = self.state()[3]
+        ks = list(self.k_buf.shape)
+        vs = list(self.v_buf.shape)
+        ks[self.seq_dim] = vis
+        vs[self.seq_dim] = vis
+        ko = torch.empty(ks, dtype=self.k_buf.dtype, device=self.k_buf.device)
+        vo = torch.empty(vs, dtype=self.v_buf.dtype, device=self.v_buf.device)
+        kd, vd = describe(ko), describe(vo)
+        with torch.cuda.device(self.k_buf.device):
+            _check(L.load().wf_kvcache_gather_logical(self._h, ctypes.byref(kd), ctypes.byref(vd),
+                                                      _stream(stream)))
+        return ko, vo

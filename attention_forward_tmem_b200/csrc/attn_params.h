@@ -1,0 +1,63 @@
+// attn_params.h -- kernel parameter block and launch table shared by the
+// attention kernels and the host runtime (internal; not part of the C ABI).
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace wf {
+
+constexpr int kBlockM = 128;     // query rows per tile (one TMEM lane per row)
+constexpr int kBlockN = 128;     // keys per KV tile
+constexpr int kThreads = 192;    // warps 0-3 softmax, warp 4 TMA, warp 5 MMA
+
+enum MaskKind : int32_t { kMaskNone = 0, kMaskCausal = 1, kMaskKeep = 2, kMaskAdd = 3 };
+enum MaskDtype : int32_t { kMaskU8 = 0, kMaskF32 = 1, kMaskBF16 = 2 };
+
+// Device status codes (same numbers as wf_status_t).
+constexpr int32_t kDevInvalidArg = 1;
+constexpr int32_t kDevTimeout = 6;
+
+// Debug switches for the bounded-wait test entry point (0 in production).
+constexpr uint32_t kDebugStarveFirstK = 1u;   // producer never loads the first K tile
+
+// Varlen schedule workspace (int32 words):
+//   [0] number of (sequence, q-tile) entries E, [1] length-check flag,
+//   [cu_q .. cu_q+B] and [cu_k .. cu_k+B] prefix sums of the lengths,
+//   [cu_t .. cu_t+B] prefix sums of q tiles per sequence,
+//   [entries ..] E pairs (sequence, q tile), longest KV range first.
+struct SchedLayout {
+  int32_t cu_q, cu_k, cu_t, entries, capacity;   // offsets in words; capacity in entries
+  int64_t words;
+};
+
+struct alignas(64) AttnParams {
+  CUtensorMap tm_q, tm_k, tm_v, tm_qr, tm_kr;   // 4-d maps (D, rows, heads, batch)
+  void *out;
+  int64_t o_sb, o_sh, o_si;                      // element strides of out (batch, head, row)
+  const void *mask;
+  int64_t m_sb, m_sh, m_si, m_sj;                // element strides of the mask (0 = broadcast)
+  int32_t mask_kind, mask_dtype;
+  int32_t batch, hq, hkv, group;
+  int32_t lq, lk;                                // dense lengths
+  int32_t varlen;
+  int32_t n_tiles_dense, nqt_dense;
+  const int32_t *ws;                             // varlen schedule (device)
+  SchedLayout sl;
+  float scale_log2;                              // qkScale * log2(e)
+  int32_t *status;                               // device status word
+  long long timeout_cycles;
+  uint32_t debug_flags;
+};
+
+using AttnLaunchFn = cudaError_t (*)(const AttnParams &, int grid, cudaStream_t);
+
+// Returns the launcher for (dtype 0 = f32 / 1 = bf16, dqk, drope, dv), or nullptr.
+AttnLaunchFn find_attn_kernel(int dtype, int dqk, int drope, int dv);
+
+cudaError_t launch_sched_prep(const int32_t *q_len, const int32_t *k_len, int32_t batch,
+                              int64_t n_q_tokens, int64_t n_k_tokens, int32_t causal,
+                              int32_t *ws, const SchedLayout &sl, int32_t *status,
+                              cudaStream_t stream);
+
+}  // namespace wf

@@ -1,0 +1,320 @@
+// kvcache.cu -- BlockKVCache: host-side rolling state and the ring-slot write.
+//
+// "Core 注意力" (WorldFoundry docs), section "Block KV cache 的调用顺序":
+// every chunk goes before_update -> update -> cached_k/cached_v ->
+// after_update; repeating the current chunk index overwrites the same logical
+// chunk, the index plus one appends or rolls the window, a skipped index is an
+// error; sink_size is a prefix that is never evicted, window_size the rolling
+// region, their sum is the cache length and divisible by chunk_size.
+//
+// Readings where the page is silent: the first index is 0; an out-of-order
+// call returns WF_ERR_ORDER and changes nothing; sink_size is a multiple of
+// chunk_size and the window holds at least one chunk; update takes exactly
+// chunk_size positions; chunk c lives in slot c while c < sink/chunk and in
+// sink/chunk + (c - sink/chunk) mod (window/chunk) afterwards.
+#include <cstdint>
+#include <cstring>
+#include <new>
+
+#include "runtime.h"
+
+using namespace wf;
+
+struct wf_kvcache {
+  wf_tensor_t k, v;     // caller-owned buffers as given
+  int32_t seq_dim;
+  int64_t chunk, sink, window, n_sink, n_window, n_slots;
+  int64_t committed, current;
+  int32_t phase;        // 0 idle, 1 before_update done, 2 update done, 3 cached done
+};
+
+namespace {
+
+enum { kIdle = 0, kBefore = 1, kUpdated = 2, kCached = 3 };
+
+int64_t slot_of(const wf_kvcache *c, int64_t idx) {
+  if (idx < c->n_sink) return idx;
+  return c->n_sink + (idx - c->n_sink) % c->n_window;
+}
+
+int64_t visible_len(const wf_kvcache *c, int64_t idx) {
+  const int64_t n = idx + 1 < c->n_slots ? idx + 1 : c->n_slots;
+  return c->chunk * n;
+}
+
+// Logical [B, H, L, D] view of a 4-d tensor whose sequence dim is seq_dim
+// (2: [B, H, L, D]; 1: [B, L, H, D]).  Strides in elements.
+struct View {
+  int64_t B, H, L, D;
+  int64_t sb, sh, sl;
+};
+View logical(const wf_tensor_t *t, int32_t seq_dim) {
+  View v;
+  v.B = t->shape[0];
+  v.sb = t->stride[0];
+  v.D = t->shape[3];
+  if (seq_dim == 2) {
+    v.H = t->shape[1]; v.sh = t->stride[1];
+    v.L = t->shape[2]; v.sl = t->stride[2];
+  } else {
+    v.L = t->shape[1]; v.sl = t->stride[1];
+    v.H = t->shape[2]; v.sh = t->stride[2];
+  }
+  return v;
+}
+
+// Copy `rows` = B*H*C rows of `row_bytes` each: source row (b, h, t) ->
+// destination row (b, h, dst_t0 + t).  `unit` bytes per thread step (16, 8, 4,
+// 2 or 1, chosen on the host so every access is aligned to it).
+template <typename U>
+__global__ void copy_rows_kernel(const uint8_t *__restrict__ src, int64_t s_b, int64_t s_h,
+                                 int64_t s_t, uint8_t *__restrict__ dst, int64_t d_b, int64_t d_h,
+                                 int64_t d_t, int64_t dst_t0, int64_t H, int64_t C, int64_t n_rows,
+                                 int64_t units_per_row) {
+  const int64_t total = n_rows * units_per_row;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = i / units_per_row, u = i - row * units_per_row;
+    const int64_t t = row % C, h = (row / C) % H, b = row / (C * H);
+    const U *s = reinterpret_cast<const U *>(src + b * s_b + h * s_h + t * s_t) + u;
+    U *d = reinterpret_cast<U *>(dst + b * d_b + h * d_h + (dst_t0 + t) * d_t) + u;
+    *d = *s;
+  }
+}
+
+int64_t gcd_pow2_unit(int64_t x) {
+  for (int64_t u = 16; u > 1; u >>= 1)
+    if (x % u == 0) return u;
+  return 1;
+}
+
+// Copy C positions of every (b, h) row from src (starting at src_t0) to dst
+// (starting at dst_t0).  Views are logical [B, H, L, D].
+wf_status_t copy_positions(const void *src_base, const View &s, int64_t src_t0, void *dst_base,
+                           const View &d, int64_t dst_t0, int64_t C, size_t es,
+                           cudaStream_t stream) {
+  const int64_t rows = s.B * s.H * C;
+  if (rows == 0 || s.D == 0) return WF_OK;
+  const int64_t row_bytes = s.D * (int64_t)es;
+  const uint8_t *src = static_cast<const uint8_t *>(src_base) + src_t0 * s.sl * (int64_t)es;
+  uint8_t *dst = static_cast<uint8_t *>(dst_base);
+  int64_t unit = gcd_pow2_unit(row_bytes);
+  const int64_t vals[] = {(int64_t)reinterpret_cast<uintptr_t>(src),
+                          (int64_t)reinterpret_cast<uintptr_t>(dst), s.sb * (int64_t)es,
+                          s.sh * (int64_t)es, s.sl * (int64_t)es, d.sb * (int64_t)es,
+                          d.sh * (int64_t)es, d.sl * (int64_t)es};
+  for (int64_t x : vals)
+    while (unit > 1 && x % unit != 0) unit >>= 1;
+  const int64_t upr = row_bytes / unit;
+  const int64_t total = rows * upr;
+  const int threads = 256;
+  int64_t blocks = (total + threads - 1) / threads;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  const int64_t sb = s.sb * es, sh = s.sh * es, st = s.sl * es;
+  const int64_t db = d.sb * es, dh = d.sh * es, dt = d.sl * es;
+  switch (unit) {
+    case 16: copy_rows_kernel<uint4><<<(int)blocks, threads, 0, stream>>>(src, sb, sh, st, dst, db, dh, dt, dst_t0, s.H, C, rows, upr); break;
+    case 8: copy_rows_kernel<uint2><<<(int)blocks, threads, 0, stream>>>(src, sb, sh, st, dst, db, dh, dt, dst_t0, s.H, C, rows, upr); break;
+    case 4: copy_rows_kernel<uint32_t><<<(int)blocks, threads, 0, stream>>>(src, sb, sh, st, dst, db, dh, dt, dst_t0, s.H, C, rows, upr); break;
+    case 2: copy_rows_kernel<uint16_t><<<(int)blocks, threads, 0, stream>>>(src, sb, sh, st, dst, db, dh, dt, dst_t0, s.H, C, rows, upr); break;
+    default: copy_rows_kernel<uint8_t><<<(int)blocks, threads, 0, stream>>>(src, sb, sh, st, dst, db, dh, dt, dst_t0, s.H, C, rows, upr); break;
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "cache copy launch");
+  return WF_OK;
+}
+
+wf_status_t check_buf(const wf_tensor_t *t, const char *name) {
+  if (!t) return fail(WF_ERR_INVALID_ARG, "%s is NULL", name);
+  if (t->ndim != 4) return fail(WF_ERR_INVALID_ARG, "%s must have 4 dims", name);
+  if (dtype_size(t->dtype) == 0) return fail(WF_ERR_INVALID_ARG, "%s: unknown dtype %d", name, t->dtype);
+  for (int i = 0; i < 4; ++i)
+    if (t->shape[i] <= 0) return fail(WF_ERR_INVALID_ARG, "%s: dim %d must be positive", name, i);
+  if (t->stride[3] != 1 && t->shape[3] > 1)
+    return fail(WF_ERR_INVALID_ARG, "%s: last dimension must be contiguous", name);
+  if (!t->data) return fail(WF_ERR_INVALID_ARG, "%s: NULL data", name);
+  return WF_OK;
+}
+
+// Same shape as the buffer except `seq_extent` positions along seq_dim.
+wf_status_t check_like(const wf_tensor_t *t, const wf_tensor_t *buf, int32_t seq_dim,
+                       int64_t seq_extent, const char *name) {
+  if (!t) return fail(WF_ERR_INVALID_ARG, "%s is NULL", name);
+  if (t->ndim != 4 || t->dtype != buf->dtype)
+    return fail(WF_ERR_INVALID_ARG, "%s: must be 4-d with the buffer's dtype", name);
+  for (int i = 0; i < 4; ++i) {
+    const int64_t want = (i == seq_dim) ? seq_extent : buf->shape[i];
+    if (t->shape[i] != want)
+      return fail(WF_ERR_INVALID_ARG, "%s: dim %d is %lld, expected %lld", name, i,
+                  (long long)t->shape[i], (long long)want);
+  }
+  if (t->stride[3] != 1 && t->shape[3] > 1)
+    return fail(WF_ERR_INVALID_ARG, "%s: last dimension must be contiguous", name);
+  if (!t->data) return fail(WF_ERR_INVALID_ARG, "%s: NULL data", name);
+  return WF_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+wf_status_t wf_kvcache_create(const wf_tensor_t *k_buf, const wf_tensor_t *v_buf, int32_t seq_dim,
+                              int64_t chunk_size, int64_t sink_size, int64_t window_size,
+                              wf_kvcache_t **out) {
+  clear_error();
+  wf_status_t st;
+  if (!out) return fail(WF_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if ((st = check_buf(k_buf, "k_buf")) != WF_OK) return st;
+  if ((st = check_buf(v_buf, "v_buf")) != WF_OK) return st;
+  if (seq_dim != 1 && seq_dim != 2) return fail(WF_ERR_INVALID_ARG, "seq_dim must be 1 or 2");
+  if (k_buf->dtype != v_buf->dtype) return fail(WF_ERR_INVALID_ARG, "k_buf and v_buf dtypes differ");
+  for (int i = 0; i < 3; ++i)
+    if (k_buf->shape[i] != v_buf->shape[i])
+      return fail(WF_ERR_INVALID_ARG, "k_buf and v_buf differ in dim %d", i);
+  const int64_t L = k_buf->shape[seq_dim];
+  if (chunk_size <= 0 || sink_size < 0 || window_size < 0)
+    return fail(WF_ERR_INVALID_ARG, "chunk_size must be positive, sink/window non-negative");
+  if (sink_size + window_size != L)
+    return fail(WF_ERR_INVALID_ARG, "sink_size + window_size (%lld) must equal the cache length %lld",
+                (long long)(sink_size + window_size), (long long)L);
+  if (L % chunk_size != 0) return fail(WF_ERR_INVALID_ARG, "cache length is not divisible by chunk_size");
+  if (sink_size % chunk_size != 0) return fail(WF_ERR_INVALID_ARG, "sink_size must be a multiple of chunk_size");
+  if (window_size < chunk_size) return fail(WF_ERR_INVALID_ARG, "the window must hold at least one chunk");
+  wf_kvcache *c = new (std::nothrow) wf_kvcache;
+  if (!c) return fail(WF_ERR_NO_MEMORY, "host allocation failed");
+  c->k = *k_buf;
+  c->v = *v_buf;
+  c->seq_dim = seq_dim;
+  c->chunk = chunk_size;
+  c->sink = sink_size;
+  c->window = window_size;
+  c->n_sink = sink_size / chunk_size;
+  c->n_window = window_size / chunk_size;
+  c->n_slots = c->n_sink + c->n_window;
+  c->committed = -1;
+  c->current = -1;
+  c->phase = kIdle;
+  *out = c;
+  return WF_OK;
+}
+
+wf_status_t wf_kvcache_before_update(wf_kvcache_t *c, int64_t idx) {
+  clear_error();
+  if (!c) return fail(WF_ERR_INVALID_ARG, "cache is NULL");
+  if (c->phase != kIdle) return fail(WF_ERR_ORDER, "before_update while chunk %lld is in progress", (long long)c->current);
+  const bool ok = c->committed < 0 ? idx == 0 : (idx == c->committed || idx == c->committed + 1);
+  if (!ok)
+    return fail(WF_ERR_ORDER, "chunk index %lld cannot follow %lld (repeat or +1 only, first is 0)",
+                (long long)idx, (long long)c->committed);
+  c->current = idx;
+  c->phase = kBefore;
+  return WF_OK;
+}
+
+wf_status_t wf_kvcache_update(wf_kvcache_t *c, const wf_tensor_t *k, const wf_tensor_t *v, void *stream) {
+  clear_error();
+  wf_status_t st;
+  if (!c) return fail(WF_ERR_INVALID_ARG, "cache is NULL");
+  if (c->phase != kBefore) return fail(WF_ERR_ORDER, "update without before_update");
+  if ((st = check_like(k, &c->k, c->seq_dim, c->chunk, "k")) != WF_OK) return st;
+  if ((st = check_like(v, &c->v, c->seq_dim, c->chunk, "v")) != WF_OK) return st;
+  const int64_t t0 = slot_of(c, c->current) * c->chunk;
+  const size_t es = dtype_size(c->k.dtype);
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if ((st = copy_positions(k->data, logical(k, c->seq_dim), 0, c->k.data, logical(&c->k, c->seq_dim),
+                           t0, c->chunk, es, cs)) != WF_OK)
+    return st;
+  if ((st = copy_positions(v->data, logical(v, c->seq_dim), 0, c->v.data, logical(&c->v, c->seq_dim),
+                           t0, c->chunk, es, cs)) != WF_OK)
+    return st;
+  c->phase = kUpdated;
+  return WF_OK;
+}
+
+static void make_view(const wf_tensor_t *buf, int32_t seq_dim, int64_t vis, wf_tensor_t *out) {
+  View lv = logical(buf, seq_dim);
+  out->data = buf->data;
+  out->dtype = buf->dtype;
+  out->ndim = 4;
+  out->shape[0] = lv.B; out->stride[0] = lv.sb;
+  out->shape[1] = lv.H; out->stride[1] = lv.sh;
+  out->shape[2] = vis;  out->stride[2] = lv.sl;
+  out->shape[3] = lv.D; out->stride[3] = buf->stride[3];
+}
+
+wf_status_t wf_kvcache_cached(wf_kvcache_t *c, wf_tensor_t *k_view, wf_tensor_t *v_view, int64_t *visible) {
+  clear_error();
+  if (!c) return fail(WF_ERR_INVALID_ARG, "cache is NULL");
+  if (c->phase != kUpdated && c->phase != kCached) return fail(WF_ERR_ORDER, "cached before update");
+  const int64_t vis = visible_len(c, c->current);
+  if (k_view) make_view(&c->k, c->seq_dim, vis, k_view);
+  if (v_view) make_view(&c->v, c->seq_dim, vis, v_view);
+  if (visible) *visible = vis;
+  c->phase = kCached;
+  return WF_OK;
+}
+
+wf_status_t wf_kvcache_after_update(wf_kvcache_t *c, int64_t idx) {
+  clear_error();
+  if (!c) return fail(WF_ERR_INVALID_ARG, "cache is NULL");
+  if (c->phase != kCached) return fail(WF_ERR_ORDER, "after_update before cached_k / cached_v");
+  if (idx != c->current)
+    return fail(WF_ERR_ORDER, "after_update(%lld) while chunk %lld is in progress", (long long)idx,
+                (long long)c->current);
+  c->committed = idx;
+  c->phase = kIdle;
+  return WF_OK;
+}
+
+wf_status_t wf_kvcache_get_state(const wf_kvcache_t *c, int64_t *cur, int64_t *committed,
+                                 int64_t *slot, int64_t *visible, int32_t *phase) {
+  clear_error();
+  if (!c) return fail(WF_ERR_INVALID_ARG, "cache is NULL");
+  if (cur) *cur = c->current;
+  if (committed) *committed = c->committed;
+  if (slot) *slot = c->current >= 0 ? slot_of(c, c->current) : -1;
+  if (visible) {
+    if (c->phase == kUpdated || c->phase == kCached) *visible = visible_len(c, c->current);
+    else *visible = c->committed >= 0 ? visible_len(c, c->committed) : 0;
+  }
+  if (phase) *phase = c->phase;
+  return WF_OK;
+}
+
+wf_status_t wf_kvcache_gather_logical(wf_kvcache_t *c, wf_tensor_t *k_out, wf_tensor_t *v_out, void *stream) {
+  clear_error();
+  wf_status_t st;
+  if (!c) return fail(WF_ERR_INVALID_ARG, "cache is NULL");
+  if (c->phase != kUpdated && c->phase != kCached) return fail(WF_ERR_ORDER, "gather before update");
+  const int64_t vis = visible_len(c, c->current);
+  if ((st = check_like(k_out, &c->k, c->seq_dim, vis, "k_out")) != WF_OK) return st;
+  if ((st = check_like(v_out, &c->v, c->seq_dim, vis, "v_out")) != WF_OK) return st;
+  const size_t es = dtype_size(c->k.dtype);
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  // logical order: sink chunks, then the window's chunks oldest first
+  const int64_t cur = c->current;
+  int64_t pos = 0;
+  auto emit = [&](int64_t idx) -> wf_status_t {
+    const int64_t src_t0 = slot_of(c, idx) * c->chunk;
+    wf_status_t s2 = copy_positions(c->k.data, logical(&c->k, c->seq_dim), src_t0, k_out->data,
+                                    logical(k_out, c->seq_dim), pos * c->chunk, c->chunk, es, cs);
+    if (s2 == WF_OK)
+      s2 = copy_positions(c->v.data, logical(&c->v, c->seq_dim), src_t0, v_out->data,
+                          logical(v_out, c->seq_dim), pos * c->chunk, c->chunk, es, cs);
+    ++pos;
+    return s2;
+  };
+  const int64_t sink_end = cur + 1 < c->n_sink ? cur + 1 : c->n_sink;
+  for (int64_t i = 0; i < sink_end; ++i)
+    if ((st = emit(i)) != WF_OK) return st;
+  int64_t first = cur - c->n_window + 1;
+  if (first < c->n_sink) first = c->n_sink;
+  for (int64_t i = first; i <= cur; ++i)
+    if ((st = emit(i)) != WF_OK) return st;
+  return WF_OK;
+}
+
+void wf_kvcache_destroy(wf_kvcache_t *c) { delete c; }
+
+}  // extern "C"

@@ -1,0 +1,465 @@
+// runtime.cu -- C ABI of the attention forward: argument checks, TMA
+// descriptors, per-device state and the launch.
+//
+// Argument set and meaning: "MLA Prefill" (CANN ATB docs), section "定义" and
+// its parameter table (Q, QRope, K, kRope, V, qSeqLen, kvSeqLen, mask,
+// headNum, qkScale, kvHeadNum, maskType, attenOut; every call returns a
+// status); dense [B, H, L, D] layout and mask meaning: "Core 注意力"
+// (WorldFoundry docs), example section.
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <string>
+#include <utility>
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "attn_params.h"
+#include "runtime.h"
+
+namespace wf {
+
+// ------------------------------------------------------------------ errors
+static thread_local std::string g_last_error;
+
+wf_status_t fail(wf_status_t st, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+void clear_error() { g_last_error.clear(); }
+
+wf_status_t cuda_fail(cudaError_t e, const char *what) {
+  return fail(WF_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+size_t dtype_size(int32_t dtype) {
+  switch (dtype) {
+    case WF_F32: return 4;
+    case WF_BF16: return 2;
+    case WF_F16: return 2;
+    case WF_U8: return 1;
+    case WF_I32: return 4;
+    default: return 0;
+  }
+}
+
+// ----------------------------------------------------------- device state
+__device__ int32_t g_device_status;   // one status word per device
+
+static std::mutex g_mu;
+static std::map<int, DeviceState> g_devices;
+static std::map<std::pair<int, cudaStream_t>, std::pair<int32_t *, size_t>> g_workspaces;
+
+DeviceState *current_device_state(wf_status_t *st) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    *st = fail(WF_ERR_NO_DEVICE, "no CUDA device: %s", cudaGetErrorString(e));
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(g_mu);
+  auto it = g_devices.find(dev);
+  if (it != g_devices.end()) return &it->second;
+  DeviceState ds;
+  if ((e = cudaDeviceGetAttribute(&ds.sm_count, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
+      (e = cudaDeviceGetAttribute(&ds.cc_major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+      (e = cudaDeviceGetAttribute(&ds.cc_minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess) {
+    *st = cuda_fail(e, "cudaDeviceGetAttribute");
+    return nullptr;
+  }
+  if (ds.cc_major != 10 || ds.cc_minor != 0) {
+    *st = fail(WF_ERR_NO_DEVICE, "device %d is sm_%d%d; this library runs on sm_100 (B200)", dev,
+               ds.cc_major, ds.cc_minor);
+    return nullptr;
+  }
+  if ((e = cudaGetSymbolAddress(reinterpret_cast<void **>(&ds.status), g_device_status)) != cudaSuccess) {
+    *st = cuda_fail(e, "cudaGetSymbolAddress(status)");
+    return nullptr;
+  }
+  return &g_devices.emplace(dev, ds).first->second;
+}
+
+// Workspace of one (device, stream): varlen schedule tables.  Calls on
+// different streams get different workspaces, so they may overlap.
+static wf_status_t stream_workspace(int dev, cudaStream_t stream, size_t bytes, int32_t **out) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  auto &slot = g_workspaces[{dev, stream}];
+  if (slot.second < bytes) {
+    if (slot.first) {
+      // the old buffer may still be read by work queued on this stream
+      cudaError_t e = cudaStreamSynchronize(stream);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+      cudaFree(slot.first);
+      slot.first = nullptr;
+      slot.second = 0;
+    }
+    size_t sz = bytes < (1u << 20) ? (1u << 20) : bytes;
+    void *p = nullptr;
+    cudaError_t e = cudaMalloc(&p, sz);
+    if (e != cudaSuccess) return fail(WF_ERR_NO_MEMORY, "cudaMalloc(%zu): %s", sz, cudaGetErrorString(e));
+    slot.first = static_cast<int32_t *>(p);
+    slot.second = sz;
+  }
+  *out = slot.first;
+  return WF_OK;
+}
+
+// ----------------------------------------------------------- TMA descriptors
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  return fn;
+}
+
+// 4-d map (D, rows, heads, batch) with a (128 B of D) x 128 rows box, 128-byte
+// swizzle, zero fill outside the tensor.  Strides in elements.
+static wf_status_t make_map(CUtensorMap *map, const void *base, int32_t dtype, int64_t d,
+                            int64_t rows, int64_t heads, int64_t batch, int64_t s_row,
+                            int64_t s_head, int64_t s_batch, const char *name) {
+  auto fn = encode_fn();
+  if (!fn) return fail(WF_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const size_t es = dtype_size(dtype);
+  const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)heads, (cuuint64_t)batch};
+  const cuuint64_t strides[3] = {(cuuint64_t)(s_row * es), (cuuint64_t)(s_head * es),
+                                 (cuuint64_t)(s_batch * es)};
+  const cuuint32_t box[4] = {(cuuint32_t)(128 / es), (cuuint32_t)kBlockM, 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUtensorMapDataType dt =
+      dtype == WF_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  CUresult r = fn(map, dt, 4, const_cast<void *>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(WF_ERR_INVALID_ARG, "%s: tensor map rejected (CUresult %d)", name, (int)r);
+  return WF_OK;
+}
+
+// ------------------------------------------------------------- validation
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static int64_t numel(const wf_tensor_t *t) {
+  int64_t n = 1;
+  for (int i = 0; i < t->ndim; ++i) n *= t->shape[i];
+  return n;
+}
+
+// Basic descriptor checks: ndim, dtype, non-negative shape, last stride 1,
+// 16-byte alignment of the base and of every other stride.
+static wf_status_t check_tensor(const wf_tensor_t *t, const char *name, int ndim, int32_t dtype,
+                                bool need_tma_layout) {
+  if (!t) return fail(WF_ERR_INVALID_ARG, "%s is NULL", name);
+  if (t->ndim != ndim) return fail(WF_ERR_INVALID_ARG, "%s: expected %d dims, got %d", name, ndim, t->ndim);
+  if (t->dtype != dtype)
+    return fail(WF_ERR_INVALID_ARG, "%s: dtype %d does not match %d", name, t->dtype, dtype);
+  for (int i = 0; i < ndim; ++i) {
+    if (t->shape[i] < 0) return fail(WF_ERR_INVALID_ARG, "%s: negative dim %d", name, i);
+    if (t->shape[i] > INT32_MAX) return fail(WF_ERR_UNSUPPORTED, "%s: dim %d above 2^31-1", name, i);
+  }
+  if (numel(t) == 0) return WF_OK;
+  if (!t->data) return fail(WF_ERR_INVALID_ARG, "%s: NULL data", name);
+  if (need_tma_layout) {
+    const size_t es = dtype_size(dtype);
+    if (t->stride[ndim - 1] != 1 && t->shape[ndim - 1] > 1)
+      return fail(WF_ERR_INVALID_ARG, "%s: last dimension must be contiguous", name);
+    if (!aligned16(t->data)) return fail(WF_ERR_INVALID_ARG, "%s: data not 16-byte aligned", name);
+    for (int i = 0; i < ndim - 1; ++i) {
+      if (t->stride[i] < 0 || (t->stride[i] * (int64_t)es) % 16 != 0)
+        return fail(WF_ERR_INVALID_ARG, "%s: stride %d is not a multiple of 16 bytes", name, i);
+      if (t->stride[i] * (int64_t)es >= (int64_t(1) << 40))
+        return fail(WF_ERR_UNSUPPORTED, "%s: stride %d too large", name, i);
+    }
+  }
+  return WF_OK;
+}
+
+struct Dims {
+  bool varlen;
+  int64_t batch, lq, lk, tq, tk, dqk, dv, drope;
+};
+
+}  // namespace wf
+
+using namespace wf;
+
+extern "C" {
+
+wf_status_t wf_attn_fwd(const wf_tensor_t *q, const wf_tensor_t *qRope, const wf_tensor_t *k,
+                        const wf_tensor_t *kRope, const wf_tensor_t *v, const wf_tensor_t *qSeqLen,
+                        const wf_tensor_t *kvSeqLen, const wf_tensor_t *mask, int32_t headNum,
+                        int32_t kvHeadNum, float qkScale, int32_t maskType, wf_tensor_t *out,
+                        void *stream) {
+  return wf_attn_fwd_debug(q, qRope, k, kRope, v, qSeqLen, kvSeqLen, mask, headNum, kvHeadNum,
+                           qkScale, maskType, out, stream, 0u, 0);
+}
+
+wf_status_t wf_attn_fwd_debug(const wf_tensor_t *q, const wf_tensor_t *qRope, const wf_tensor_t *k,
+                              const wf_tensor_t *kRope, const wf_tensor_t *v,
+                              const wf_tensor_t *qSeqLen, const wf_tensor_t *kvSeqLen,
+                              const wf_tensor_t *mask, int32_t headNum, int32_t kvHeadNum,
+                              float qkScale, int32_t maskType, wf_tensor_t *out, void *stream,
+                              uint32_t debug_flags, int64_t timeout_cycles) {
+  clear_error();
+  wf_status_t st;
+  if (!q || !k || !v || !out) return fail(WF_ERR_INVALID_ARG, "q, k, v and out are required");
+  const int32_t dt = q->dtype;
+  if (dt != WF_BF16 && dt != WF_F32)
+    return fail(WF_ERR_UNSUPPORTED, "q dtype %d: only WF_BF16 and WF_F32 are implemented", dt);
+  if (maskType < WF_MASK_NONE || maskType > WF_MASK_ADDITIVE)
+    return fail(WF_ERR_INVALID_ARG, "maskType %d out of range", maskType);
+  if (!std::isfinite(qkScale)) return fail(WF_ERR_INVALID_ARG, "qkScale is not finite");
+  if ((qSeqLen == nullptr) != (kvSeqLen == nullptr))
+    return fail(WF_ERR_INVALID_ARG, "qSeqLen and kvSeqLen are given together or not at all");
+  if ((qRope == nullptr) != (kRope == nullptr))
+    return fail(WF_ERR_INVALID_ARG, "qRope and kRope are given together or not at all");
+  if (headNum <= 0 || kvHeadNum <= 0 || headNum % kvHeadNum != 0)
+    return fail(WF_ERR_INVALID_ARG, "headNum %d must be a positive multiple of kvHeadNum %d", headNum,
+                kvHeadNum);
+
+  Dims d{};
+  d.varlen = qSeqLen != nullptr;
+  const int nd = d.varlen ? 3 : 4;
+  if ((st = check_tensor(q, "q", nd, dt, true)) != WF_OK) return st;
+  if ((st = check_tensor(k, "k", nd, dt, true)) != WF_OK) return st;
+  if ((st = check_tensor(v, "v", nd, dt, true)) != WF_OK) return st;
+  if ((st = check_tensor(out, "out", nd, dt, true)) != WF_OK) return st;
+  const int hd = nd - 2;   // head dim index: 1 in both layouts
+  const int rd = d.varlen ? 0 : 2;   // row (sequence) dim index
+  if (q->shape[1] != headNum || out->shape[1] != headNum)
+    return fail(WF_ERR_INVALID_ARG, "q/out head dim must equal headNum %d", headNum);
+  if (k->shape[1] != kvHeadNum || v->shape[1] != kvHeadNum)
+    return fail(WF_ERR_INVALID_ARG, "k/v head dim must equal kvHeadNum %d", kvHeadNum);
+  (void)hd;
+  d.dqk = q->shape[nd - 1];
+  d.dv = v->shape[nd - 1];
+  if (k->shape[nd - 1] != d.dqk) return fail(WF_ERR_INVALID_ARG, "q and k head sizes differ");
+  if (out->shape[nd - 1] != d.dv) return fail(WF_ERR_INVALID_ARG, "out and v head sizes differ");
+  if (k->shape[rd] != v->shape[rd]) return fail(WF_ERR_INVALID_ARG, "k and v lengths differ");
+  if (out->shape[rd] != q->shape[rd]) return fail(WF_ERR_INVALID_ARG, "out and q lengths differ");
+  if (!d.varlen) {
+    d.batch = q->shape[0];
+    if (k->shape[0] != d.batch || v->shape[0] != d.batch || out->shape[0] != d.batch)
+      return fail(WF_ERR_INVALID_ARG, "batch sizes differ");
+    d.lq = q->shape[2];
+    d.lk = k->shape[2];
+  } else {
+    if ((st = check_tensor(qSeqLen, "qSeqLen", 1, WF_I32, false)) != WF_OK) return st;
+    if ((st = check_tensor(kvSeqLen, "kvSeqLen", 1, WF_I32, false)) != WF_OK) return st;
+    if (qSeqLen->shape[0] != kvSeqLen->shape[0])
+      return fail(WF_ERR_INVALID_ARG, "qSeqLen and kvSeqLen have different lengths");
+    if (qSeqLen->shape[0] > 0 && (qSeqLen->stride[0] != 1 || kvSeqLen->stride[0] != 1))
+      return fail(WF_ERR_INVALID_ARG, "qSeqLen / kvSeqLen must be contiguous");
+    d.batch = qSeqLen->shape[0];
+    d.tq = q->shape[0];
+    d.tk = k->shape[0];
+  }
+  d.drope = 0;
+  if (qRope) {
+    if ((st = check_tensor(qRope, "qRope", nd, dt, true)) != WF_OK) return st;
+    if ((st = check_tensor(kRope, "kRope", nd, dt, true)) != WF_OK) return st;
+    d.drope = qRope->shape[nd - 1];
+    if (kRope->shape[nd - 1] != d.drope) return fail(WF_ERR_INVALID_ARG, "qRope/kRope sizes differ");
+    for (int i = 0; i < nd - 1; ++i) {
+      if (qRope->shape[i] != q->shape[i]) return fail(WF_ERR_INVALID_ARG, "qRope shape does not match q");
+      if (kRope->shape[i] != k->shape[i]) return fail(WF_ERR_INVALID_ARG, "kRope shape does not match k");
+    }
+  }
+
+  // mask
+  const bool explicit_mask = maskType == WF_MASK_BOOL_KEEP || maskType == WF_MASK_ADDITIVE;
+  if (!explicit_mask && mask) return fail(WF_ERR_INVALID_ARG, "mask given but maskType is %d", maskType);
+  int64_t ms[4] = {0, 0, 0, 0};
+  int32_t mask_dtype = kMaskU8;
+  if (explicit_mask) {
+    if (d.varlen)
+      return fail(WF_ERR_UNSUPPORTED, "explicit masks are supported in the dense layout only");
+    if (!mask) return fail(WF_ERR_INVALID_ARG, "maskType %d needs a mask tensor", maskType);
+    if (mask->ndim != 4) return fail(WF_ERR_INVALID_ARG, "mask must have 4 dims [B|1, H|1, Lq, Lk]");
+    if (maskType == WF_MASK_BOOL_KEEP) {
+      if (mask->dtype != WF_U8) return fail(WF_ERR_INVALID_ARG, "bool keep-mask dtype must be WF_U8");
+      mask_dtype = kMaskU8;
+    } else {
+      if (mask->dtype == WF_F32) mask_dtype = kMaskF32;
+      else if (mask->dtype == WF_BF16 && dt == WF_BF16) mask_dtype = kMaskBF16;
+      else return fail(WF_ERR_INVALID_ARG, "additive mask dtype must be WF_F32 (or WF_BF16 with bf16 q)");
+    }
+    const int64_t full[4] = {d.batch, headNum, d.lq, d.lk};
+    for (int i = 0; i < 4; ++i) {
+      if (mask->shape[i] == full[i]) ms[i] = mask->stride[i];
+      else if (mask->shape[i] == 1) ms[i] = 0;
+      else return fail(WF_ERR_INVALID_ARG, "mask dim %d is %lld, expected %lld or 1", i,
+                       (long long)mask->shape[i], (long long)full[i]);
+      if (full[i] > 1 && mask->shape[i] == full[i] && ms[i] < 0)
+        return fail(WF_ERR_INVALID_ARG, "mask stride %d is negative", i);
+    }
+    if (numel(mask) > 0 && !mask->data) return fail(WF_ERR_INVALID_ARG, "mask: NULL data");
+  }
+
+  // supported head sizes
+  if (d.drope && !(d.drope == 64 && d.dqk == 128 && d.dv == 128 && dt == WF_BF16))
+    return fail(WF_ERR_UNSUPPORTED, "rope part needs bf16, Dqk = Dv = 128 and a 64-wide rope");
+  AttnLaunchFn launch = find_attn_kernel(dt == WF_BF16 ? 1 : 0, (int)d.dqk, (int)d.drope, (int)d.dv);
+  if (!launch)
+    return fail(WF_ERR_UNSUPPORTED, "head sizes Dqk=%lld Dv=%lld (rope %lld) are not implemented",
+                (long long)d.dqk, (long long)d.dv, (long long)d.drope);
+
+  // nothing to compute?
+  if (d.batch == 0 || numel(q) == 0) return WF_OK;
+
+  DeviceState *ds = current_device_state(&st);
+  if (!ds) return st;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+
+  AttnParams p;
+  std::memset(&p, 0, sizeof(p));
+  const int64_t es = (int64_t)dtype_size(dt);
+  (void)es;
+  // q / k / v maps: (D, rows, heads, batch)
+  if (!d.varlen) {
+    st = make_map(&p.tm_q, q->data, dt, d.dqk, d.lq, headNum, d.batch, q->stride[2], q->stride[1], q->stride[0], "q");
+    if (st == WF_OK)
+      st = make_map(&p.tm_k, k->data, dt, d.dqk, d.lk > 0 ? d.lk : 1, kvHeadNum, d.batch, k->stride[2], k->stride[1], k->stride[0], "k");
+    if (st == WF_OK)
+      st = make_map(&p.tm_v, v->data, dt, d.dv, d.lk > 0 ? d.lk : 1, kvHeadNum, d.batch, v->stride[2], v->stride[1], v->stride[0], "v");
+    if (st == WF_OK && d.drope) {
+      st = make_map(&p.tm_qr, qRope->data, dt, d.drope, d.lq, headNum, d.batch, qRope->stride[2], qRope->stride[1], qRope->stride[0], "qRope");
+      if (st == WF_OK)
+        st = make_map(&p.tm_kr, kRope->data, dt, d.drope, d.lk > 0 ? d.lk : 1, kvHeadNum, d.batch, kRope->stride[2], kRope->stride[1], kRope->stride[0], "kRope");
+    }
+  } else {
+    const int64_t tk = d.tk > 0 ? d.tk : 1;
+    st = make_map(&p.tm_q, q->data, dt, d.dqk, d.tq, headNum, 1, q->stride[0], q->stride[1], q->stride[0] * d.tq, "q");
+    if (st == WF_OK)
+      st = make_map(&p.tm_k, k->data, dt, d.dqk, tk, kvHeadNum, 1, k->stride[0], k->stride[1], k->stride[0] * tk, "k");
+    if (st == WF_OK)
+      st = make_map(&p.tm_v, v->data, dt, d.dv, tk, kvHeadNum, 1, v->stride[0], v->stride[1], v->stride[0] * tk, "v");
+    if (st == WF_OK && d.drope) {
+      st = make_map(&p.tm_qr, qRope->data, dt, d.drope, d.tq, headNum, 1, qRope->stride[0], qRope->stride[1], qRope->stride[0] * d.tq, "qRope");
+      if (st == WF_OK)
+        st = make_map(&p.tm_kr, kRope->data, dt, d.drope, tk, kvHeadNum, 1, kRope->stride[0], kRope->stride[1], kRope->stride[0] * tk, "kRope");
+    }
+  }
+  if (st != WF_OK) return st;
+  if (!d.drope) {   // unused maps: copies of q / k so the descriptor is well formed
+    p.tm_qr = p.tm_q;
+    p.tm_kr = p.tm_k;
+  }
+
+  p.out = out->data;
+  if (!d.varlen) {
+    p.o_sb = out->stride[0];
+    p.o_sh = out->stride[1];
+    p.o_si = out->stride[2];
+  } else {
+    p.o_sb = 0;
+    p.o_sh = out->stride[1];
+    p.o_si = out->stride[0];
+  }
+  p.mask = explicit_mask ? mask->data : nullptr;
+  p.m_sb = ms[0];
+  p.m_sh = ms[1];
+  p.m_si = ms[2];
+  p.m_sj = ms[3];
+  p.mask_kind = maskType;
+  p.mask_dtype = mask_dtype;
+  p.batch = (int32_t)d.batch;
+  p.hq = headNum;
+  p.hkv = kvHeadNum;
+  p.group = headNum / kvHeadNum;
+  p.varlen = d.varlen ? 1 : 0;
+  p.scale_log2 = qkScale * 1.4426950408889634f;
+  p.status = ds->status;
+  p.timeout_cycles = timeout_cycles > 0 ? timeout_cycles : (2LL << 30);
+  p.debug_flags = debug_flags;
+
+  int grid = ds->sm_count;
+  if (!d.varlen) {
+    p.lq = (int32_t)d.lq;
+    p.lk = (int32_t)d.lk;
+    const int64_t nqt = (d.lq + kBlockM - 1) / kBlockM;
+    const int64_t tiles = nqt * d.batch * headNum;
+    if (tiles > INT32_MAX) return fail(WF_ERR_UNSUPPORTED, "too many tiles (%lld)", (long long)tiles);
+    p.nqt_dense = (int32_t)nqt;
+    p.n_tiles_dense = (int32_t)tiles;
+    if (tiles < grid) grid = (int)tiles;
+  } else {
+    // schedule workspace
+    const int64_t B = d.batch;
+    const int64_t cap = (d.tq + kBlockM - 1) / kBlockM + B;
+    if (cap * headNum > INT32_MAX) return fail(WF_ERR_UNSUPPORTED, "too many tiles");
+    SchedLayout sl;
+    sl.cu_q = 2;
+    sl.cu_k = (int32_t)(sl.cu_q + B + 1);
+    sl.cu_t = (int32_t)(sl.cu_k + B + 1);
+    sl.entries = (int32_t)(((sl.cu_t + B + 1) + 3) & ~int64_t(3));
+    sl.capacity = (int32_t)cap;
+    sl.words = sl.entries + 2 * cap;
+    int32_t *ws = nullptr;
+    if ((st = stream_workspace(dev, cs, (size_t)sl.words * 4, &ws)) != WF_OK) return st;
+    cudaError_t e = launch_sched_prep(static_cast<const int32_t *>(qSeqLen->data),
+                                      static_cast<const int32_t *>(kvSeqLen->data), (int32_t)B,
+                                      d.tq, d.tk, maskType == WF_MASK_CAUSAL ? 1 : 0, ws, sl,
+                                      ds->status, cs);
+    if (e != cudaSuccess) return cuda_fail(e, "sched_prep launch");
+    p.ws = ws;
+    p.sl = sl;
+  }
+  cudaError_t e = launch(p, grid, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "attention kernel launch");
+  return WF_OK;
+}
+
+wf_status_t wf_get_device_status(void *stream) {
+  clear_error();
+  wf_status_t st;
+  DeviceState *ds = current_device_state(&st);
+  if (!ds) return st;
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int32_t v = 0;
+  if ((e = cudaMemcpy(&v, ds->status, sizeof(v), cudaMemcpyDeviceToHost)) != cudaSuccess)
+    return cuda_fail(e, "reading the device status");
+  const int32_t zero = 0;
+  if ((e = cudaMemcpy(ds->status, &zero, sizeof(zero), cudaMemcpyHostToDevice)) != cudaSuccess)
+    return cuda_fail(e, "clearing the device status");
+  if (v == kDevTimeout) return fail(WF_ERR_TIMEOUT, "a bounded device wait ran out");
+  if (v == kDevInvalidArg) return fail(WF_ERR_INVALID_ARG, "device-side length check failed");
+  if (v != 0) return fail(WF_ERR_CUDA, "device status %d", v);
+  return WF_OK;
+}
+
+const char *wf_last_error_message(void) { return g_last_error.c_str(); }
+
+int32_t wf_version(void) { return WF_ATTN_VERSION; }
+
+void wf_shutdown(void) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  int cur = 0;
+  cudaGetDevice(&cur);
+  for (auto &kv : g_workspaces) {
+    if (kv.second.first) {
+      cudaSetDevice(kv.first.first);
+      cudaFree(kv.second.first);
+    }
+  }
+  g_workspaces.clear();
+  cudaSetDevice(cur);
+}
+
+}  // extern "C"

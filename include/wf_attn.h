@@ -136,6 +136,26 @@ wf_status_t wf_attn_fwd(const wf_tensor_t *q, const wf_tensor_t *qRope,
                         int32_t headNum, int32_t kvHeadNum, float qkScale,
                         int32_t maskType, wf_tensor_t *out, void *stream);
 
+/*
+ * wf_attn_fwd_debug -- wf_attn_fwd with test switches for the bounded waits
+ * (no counterpart on the pages; a diagnostic aid).
+ *   debug_flags bit 0: the kernel's copy engine never loads the first K tile,
+ *     so the matrix-multiply stage's bounded wait runs out.  The call still
+ *     returns WF_OK; wf_get_device_status() then reports WF_ERR_TIMEOUT and
+ *     the device stays usable.  `out` is undefined after a timeout.
+ *   timeout_cycles: bound of every device wait in SM clock cycles; 0 selects
+ *     the production bound (2^31 cycles, about one second).
+ * With debug_flags = 0 and timeout_cycles = 0 this is exactly wf_attn_fwd.
+ */
+wf_status_t wf_attn_fwd_debug(const wf_tensor_t *q, const wf_tensor_t *qRope,
+                              const wf_tensor_t *k, const wf_tensor_t *kRope,
+                              const wf_tensor_t *v,
+                              const wf_tensor_t *qSeqLen, const wf_tensor_t *kvSeqLen,
+                              const wf_tensor_t *mask,
+                              int32_t headNum, int32_t kvHeadNum, float qkScale,
+                              int32_t maskType, wf_tensor_t *out, void *stream,
+                              uint32_t debug_flags, int64_t timeout_cycles);
+
 /* ---------------------------------------------------------------------------
  * BlockKVCache ([P1] "Block KV cache 的调用顺序").
  *

@@ -1,0 +1,207 @@
+"""The C-ABI library on the host (no GPU): it loads, exports every declared
+symbol, rejects bad arguments before touching a device, and enforces the
+BlockKVCache call order."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+from attention_forward_tmem_b200 import _lib as L
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+ALIGNED = 0x10000          # fake, 16-byte aligned addresses: never dereferenced on the host
+
+
+def _declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        for m in re.finditer(r"\b(wf_[a-z_0-9]+)\s*\(", src):
+            names.add(m.group(1))
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return L.load()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    declared = _declared_functions()
+    assert "wf_attn_fwd" in declared and "wf_kvcache_update" in declared
+    for name in declared:
+        assert hasattr(lib, name), f"{name} is declared in include/ but not exported"
+    assert set(L.SIGNATURES) >= declared
+
+
+def test_version(lib):
+    assert lib.wf_version() == 1
+
+
+def _t(shape, dtype=L.WF_BF16, data=ALIGNED, strides=None):
+    d = L.WfTensor()
+    d.data = data
+    d.dtype = dtype
+    d.ndim = len(shape)
+    if strides is None:
+        strides, acc = [], 1
+        for s in reversed(shape):
+            strides.insert(0, acc)
+            acc *= s
+    for i, (s, st) in enumerate(zip(shape, strides)):
+        d.shape[i] = s
+        d.stride[i] = st
+    return d
+
+
+def _call(lib, q, k, v, out, *, qr=None, kr=None, ql=None, kl=None, mask=None, hq=None, hk=None,
+          scale=0.125, mt=L.WF_MASK_NONE):
+    r = lambda x: ctypes.byref(x) if x is not None else None
+    hq = q.shape[1] if hq is None else hq
+    hk = k.shape[1] if hk is None else hk
+    return lib.wf_attn_fwd(r(q), r(qr), r(k), r(kr), r(v), r(ql), r(kl), r(mask), hq, hk, scale, mt,
+                           ctypes.byref(out), None)
+
+
+def _dense(B=2, Hq=8, Hk=2, Lq=100, Lk=120, D=128, Dv=128, dtype=L.WF_BF16):
+    return (_t([B, Hq, Lq, D], dtype), _t([B, Hk, Lk, D], dtype), _t([B, Hk, Lk, Dv], dtype),
+            _t([B, Hq, Lq, Dv], dtype))
+
+
+def test_valid_call_reaches_device_check(lib):
+    """Everything valid: the only thing left to fail on a CPU host is the device."""
+    q, k, v, o = _dense()
+    st = _call(lib, q, k, v, o, mt=L.WF_MASK_CAUSAL)
+    assert st in (L.WF_ERR_NO_DEVICE, L.WF_OK)   # WF_OK only where a B200 is present
+
+
+@pytest.mark.parametrize("case,expect", [
+    ("f16", L.WF_ERR_UNSUPPORTED),
+    ("heads_not_divisible", L.WF_ERR_INVALID_ARG),
+    ("head_count_mismatch", L.WF_ERR_INVALID_ARG),
+    ("dtype_mix", L.WF_ERR_INVALID_ARG),
+    ("dv_unsupported", L.WF_ERR_UNSUPPORTED),
+    ("unaligned_ptr", L.WF_ERR_INVALID_ARG),
+    ("unaligned_stride", L.WF_ERR_INVALID_ARG),
+    ("noncontig_last", L.WF_ERR_INVALID_ARG),
+    ("mask_missing", L.WF_ERR_INVALID_ARG),
+    ("mask_with_causal", L.WF_ERR_INVALID_ARG),
+    ("mask_with_varlen", L.WF_ERR_UNSUPPORTED),
+    ("mask_bad_shape", L.WF_ERR_INVALID_ARG),
+    ("mask_bad_dtype", L.WF_ERR_INVALID_ARG),
+    ("rope_one_side", L.WF_ERR_INVALID_ARG),
+    ("rope_bad_width", L.WF_ERR_UNSUPPORTED),
+    ("seqlen_one_side", L.WF_ERR_INVALID_ARG),
+    ("seqlen_len_mismatch", L.WF_ERR_INVALID_ARG),
+    ("bad_mask_type", L.WF_ERR_INVALID_ARG),
+    ("nan_scale", L.WF_ERR_INVALID_ARG),
+    ("batch_mismatch", L.WF_ERR_INVALID_ARG),
+])
+def test_argument_errors(lib, case, expect):
+    q, k, v, o = _dense()
+    kw = {}
+    if case == "f16":
+        q, k, v, o = _dense(dtype=L.WF_F16)
+    elif case == "heads_not_divisible":
+        q, k, v, o = _dense(Hq=6, Hk=4)
+    elif case == "head_count_mismatch":
+        kw["hq"] = 4
+    elif case == "dtype_mix":
+        v = _t([2, 2, 120, 128], L.WF_F32)
+    elif case == "dv_unsupported":
+        q, k, v, o = _dense(Dv=80)
+    elif case == "unaligned_ptr":
+        q = _t([2, 8, 100, 128], data=ALIGNED + 2)
+    elif case == "unaligned_stride":
+        q = _t([2, 8, 100, 128], strides=[8 * 100 * 132, 100 * 132, 132 - 4 + 1, 1])
+    elif case == "noncontig_last":
+        q = _t([2, 8, 100, 128], strides=[8 * 100 * 256, 100 * 256, 256, 2])
+    elif case == "mask_missing":
+        kw["mt"] = L.WF_MASK_BOOL_KEEP
+    elif case == "mask_with_causal":
+        kw.update(mt=L.WF_MASK_CAUSAL, mask=_t([2, 8, 100, 120], L.WF_U8))
+    elif case == "mask_with_varlen":
+        q, k, v, o = _t([300, 8, 128]), _t([300, 2, 128]), _t([300, 2, 128]), _t([300, 8, 128])
+        kw.update(ql=_t([3], L.WF_I32), kl=_t([3], L.WF_I32), mask=_t([1, 1, 300, 300], L.WF_U8),
+                  mt=L.WF_MASK_BOOL_KEEP)
+    elif case == "mask_bad_shape":
+        kw.update(mt=L.WF_MASK_BOOL_KEEP, mask=_t([2, 3, 100, 120], L.WF_U8))
+    elif case == "mask_bad_dtype":
+        kw.update(mt=L.WF_MASK_BOOL_KEEP, mask=_t([2, 8, 100, 120], L.WF_F32))
+    elif case == "rope_one_side":
+        kw.update(qr=_t([2, 8, 100, 64]))
+    elif case == "rope_bad_width":
+        kw.update(qr=_t([2, 8, 100, 32]), kr=_t([2, 2, 120, 32]))
+    elif case == "seqlen_one_side":
+        q, k, v, o = _t([300, 8, 128]), _t([300, 2, 128]), _t([300, 2, 128]), _t([300, 8, 128])
+        kw.update(ql=_t([3], L.WF_I32))
+    elif case == "seqlen_len_mismatch":
+        q, k, v, o = _t([300, 8, 128]), _t([300, 2, 128]), _t([300, 2, 128]), _t([300, 8, 128])
+        kw.update(ql=_t([3], L.WF_I32), kl=_t([4], L.WF_I32))
+    elif case == "bad_mask_type":
+        kw["mt"] = 7
+    elif case == "nan_scale":
+        kw["scale"] = float("nan")
+    elif case == "batch_mismatch":
+        k = _t([3, 2, 120, 128])
+    assert _call(lib, q, k, v, o, **kw) == expect
+    assert lib.wf_last_error_message()
+
+
+def test_empty_input_is_a_no_op(lib):
+    q, k, v, o = _dense(Lq=0)
+    q.data = None
+    o.data = None
+    assert _call(lib, q, k, v, o) == L.WF_OK
+
+
+# ------------------------------------------------------------------ BlockKVCache
+
+def _cache(lib, L_=8, chunk=2, window=6, sink=2, seq_dim=2):
+    shape = [1, 2, L_, 4] if seq_dim == 2 else [1, L_, 2, 4]
+    h = ctypes.c_void_p()
+    st = lib.wf_kvcache_create(ctypes.byref(_t(shape, L.WF_F32)), ctypes.byref(_t(shape, L.WF_F32)),
+                               seq_dim, chunk, sink, window, ctypes.byref(h))
+    return st, h
+
+
+@pytest.mark.parametrize("L_,chunk,window,sink", [(8, 3, 8, 0), (8, 2, 4, 2), (8, 4, 6, 2),
+                                                  (8, 2, 0, 8), (8, 0, 8, 0)])
+def test_cache_bad_sizes(lib, L_, chunk, window, sink):
+    st, h = _cache(lib, L_, chunk, window, sink)
+    assert st == L.WF_ERR_INVALID_ARG and not h.value
+
+
+def test_cache_order_errors_on_host(lib):
+    st, h = _cache(lib)
+    assert st == L.WF_OK
+    state = lambda: _state(lib, h)
+    s0 = state()
+    assert s0 == (-1, -1, -1, 0, 0)
+    assert lib.wf_kvcache_before_update(h, 1) == L.WF_ERR_ORDER        # first must be 0
+    assert state() == s0
+    kv = _t([1, 2, 2, 4], L.WF_F32)
+    assert lib.wf_kvcache_update(h, ctypes.byref(kv), ctypes.byref(kv), None) == L.WF_ERR_ORDER
+    assert lib.wf_kvcache_cached(h, None, None, None) == L.WF_ERR_ORDER
+    assert lib.wf_kvcache_after_update(h, 0) == L.WF_ERR_ORDER
+    assert state() == s0
+    assert lib.wf_kvcache_before_update(h, 0) == L.WF_OK
+    assert state() == (0, -1, 0, 0, 1)
+    assert lib.wf_kvcache_before_update(h, 0) == L.WF_ERR_ORDER        # twice
+    assert lib.wf_kvcache_cached(h, None, None, None) == L.WF_ERR_ORDER  # before update
+    assert lib.wf_kvcache_after_update(h, 0) == L.WF_ERR_ORDER         # before cached
+    bad = _t([1, 2, 3, 4], L.WF_F32)                                   # not chunk_size positions
+    assert lib.wf_kvcache_update(h, ctypes.byref(bad), ctypes.byref(bad), None) == L.WF_ERR_INVALID_ARG
+    assert state() == (0, -1, 0, 0, 1)
+    lib.wf_kvcache_destroy(h)
+
+
+def _state(lib, h):
+    cur, com, slot, vis = (ctypes.c_int64() for _ in range(4))
+    ph = ctypes.c_int32()
+    assert lib.wf_kvcache_get_state(h, ctypes.byref(cur), ctypes.byref(com), ctypes.byref(slot),
+                                    ctypes.byref(vis), ctypes.byref(ph)) == L.WF_OK
+    return cur.value, com.value, slot.value, vis.value, ph.value
