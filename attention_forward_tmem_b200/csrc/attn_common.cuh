@@ -1,0 +1,299 @@
+// attn_common.cuh -- pieces shared by the attention kernels: work-unit to
+// tile mapping, bounded mbarrier waits, the online-softmax step of one score
+// row and the output store.
+//
+// The softmax follows the definition of "Core 注意力" (WorldFoundry docs,
+// example section: a bool mask keeps scores, a float mask is added to them)
+// and "MLA Prefill" (CANN ATB docs, parameter table: qkScale multiplies
+// Q*K^T); it is evaluated online in the log2 domain:
+//   x_j = s_j * qkScale * log2(e) (+ mask_j * log2(e)),  masked x_j = -inf,
+//   m   = running max,  p_j = 2^(x_j - m),  l = running sum of p,
+//   out = (sum_j p_j v_j) / l.
+// The running max is only raised when a row's new max exceeds it by more
+// than 2^8 ("lazy rescale"); p_j then stays below 2^8 and the final division
+// by l cancels the stale max exactly.
+#pragma once
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "attn_params.h"
+#include "sm100_ptx.cuh"
+
+namespace wf {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescaleThreshold = 8.0f;   // log2 units
+
+
+struct TileInfo {
+  int32_t b, h, hk, q0, lq, lk, qrow, krow, n_kv, off, tma_b;
+};
+
+// Sub-tile `sub` (128 rows each) of work unit `t`.  Dense units are ordered
+// longest causal range first; packed units come from the schedule table.
+__device__ __forceinline__ TileInfo tile_info(const AttnParams &p, int32_t t, int32_t sub) {
+  TileInfo ti;
+  int32_t u;
+  if (!p.varlen) {
+    const int32_t bh = p.batch * p.hq;
+    u = p.units_per_bh - 1 - t / bh;
+    const int32_t r = t % bh;
+    ti.b = r / p.hq;
+    ti.h = r % p.hq;
+    ti.lq = p.lq;
+    ti.lk = p.lk;
+    ti.krow = 0;
+    ti.tma_b = ti.b;
+    ti.q0 = u * p.unit_rows + sub * kBlockM;
+    ti.qrow = ti.q0;
+  } else {
+    const int32_t e = t / p.hq;
+    ti.h = t % p.hq;
+    const int32_t *ent = p.ws + p.sl.entries + 2 * e;
+    ti.b = __ldg(ent);
+    u = __ldg(ent + 1);
+    const int32_t cq = __ldg(p.ws + p.sl.cu_q + ti.b), ck = __ldg(p.ws + p.sl.cu_k + ti.b);
+    ti.lq = __ldg(p.ws + p.sl.cu_q + ti.b + 1) - cq;
+    ti.lk = __ldg(p.ws + p.sl.cu_k + ti.b + 1) - ck;
+    ti.krow = ck;
+    ti.tma_b = 0;
+    ti.q0 = u * p.unit_rows + sub * kBlockM;
+    ti.qrow = cq + ti.q0;
+  }
+  ti.hk = ti.h / p.group;
+  ti.off = ti.lk - ti.lq;
+  int32_t kend = ti.q0 < ti.lq ? ti.lk : 0;            // no valid row: nothing to do
+  if (p.mask_kind == kMaskCausal) {
+    const int32_t last = min(ti.q0 + kBlockM, ti.lq);   // one past the last valid row
+    kend = min(kend, last + ti.off);
+  }
+  ti.n_kv = kend > 0 ? (kend + kBlockN - 1) / kBlockN : 0;
+  return ti;
+}
+
+__device__ __forceinline__ int32_t num_units(const AttnParams &p) {
+  if (!p.varlen) return p.n_units_dense;
+  return __ldg(p.ws) * p.hq;
+}
+
+// Bounded wait.  Returns false (and raises the CTA abort flag) on expiry, or
+// if another role already aborted.
+__device__ __forceinline__ bool bwait(uint64_t *bar, uint32_t parity, volatile int32_t *abort,
+                                      const AttnParams &p) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (clock64() - t0 > p.timeout_cycles) {
+      *abort = 1;
+      atomicCAS(p.status, 0, kDevTimeout);
+      return false;
+    }
+  }
+}
+
+// Wait used while draining after an abort: ignores the abort flag, still bounded.
+__device__ __forceinline__ bool drain_wait(uint64_t *bar, uint32_t parity, const AttnParams &p) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > p.timeout_cycles) {
+      atomicCAS(p.status, 0, kDevTimeout);
+      return false;
+    }
+  }
+  return true;
+}
+
+// Last fill index the producer issued per barrier (-1: none), for the drain.
+struct ProducerLog {
+  int32_t q_last;
+  int32_t k_last[3], v_last[3];
+};
+
+// One softmax step of one score row (128 keys starting at k0).  `sr` holds the
+// raw fp32 scores; on return `x` holds p_j (0 for masked keys), m / l are
+// updated, and the return value is the factor O must be multiplied by
+// (1 when the running max did not move).
+// kEmuPer16: of every 16 score columns, this many are exponentiated on the FMA
+// pipe (exp2_poly2) instead of the MUFU unit, in tiles without masked scores.
+// At head size 128 the MUFU rate alone (16 per clock per SM) makes one
+// tile's softmax as long as the other tile's two MMAs.
+template <int kEmuPer16>
+__device__ __forceinline__ float softmax_row(const AttnParams &p, const TileInfo &ti, int32_t row,
+                                             int32_t k0, const uint32_t (&sr)[128],
+                                             float (&x)[128], float &m, float &l) {
+  const bool causal = p.mask_kind == kMaskCausal;
+  const bool explicit_mask = p.mask_kind == kMaskKeep || p.mask_kind == kMaskAdd;
+  const bool row_valid = row < ti.lq;
+  int32_t lim = ti.lk - 1 - k0;                      // last visible column of this row
+  if (causal) lim = min(lim, row + ti.off - k0);
+  const bool need_mask = (k0 + kBlockN > ti.lk) || (causal && (k0 + kBlockN - 1 > ti.q0 + ti.off));
+  // prescaled: x holds scaled scores after the first pass (explicit masks, or a
+  // non-positive scale for which max and scaling do not commute)
+  const bool prescaled = explicit_mask || !(p.scale_log2 > 0.f);
+  // pass 1: x = (masked) scores, and their max in four independent chains of
+  // three-input max.
+  if (!prescaled) {
+    if (need_mask) {
+#pragma unroll
+      for (int c = 0; c < 128; ++c) x[c] = (c <= lim) ? __uint_as_float(sr[c]) : -INFINITY;
+    } else {
+#pragma unroll
+      for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(sr[c]);
+    }
+  } else if (!explicit_mask) {
+#pragma unroll
+    for (int c = 0; c < 128; ++c)
+      x[c] = (c <= lim) ? __uint_as_float(sr[c]) * p.scale_log2 : -INFINITY;
+  } else {
+    const int64_t mrow = (int64_t)ti.b * p.m_sb + (int64_t)ti.h * p.m_sh + (int64_t)row * p.m_si;
+    if (p.mask_kind == kMaskKeep) {
+      const uint8_t *mp = reinterpret_cast<const uint8_t *>(p.mask) + mrow;
+#pragma unroll
+      for (int c = 0; c < 128; ++c) {
+        const bool keep = row_valid && c <= lim && mp[(int64_t)(k0 + c) * p.m_sj] != 0;
+        x[c] = keep ? __uint_as_float(sr[c]) * p.scale_log2 : -INFINITY;
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < 128; ++c) {
+        float add = 0.f;
+        const bool in = row_valid && c <= lim;
+        if (in) {
+          const int64_t idx = mrow + (int64_t)(k0 + c) * p.m_sj;
+          add = p.mask_dtype == kMaskF32
+                    ? reinterpret_cast<const float *>(p.mask)[idx]
+                    : __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(p.mask)[idx]);
+        }
+        x[c] = in ? fmaf(add, kLog2e, __uint_as_float(sr[c]) * p.scale_log2) : -INFINITY;
+      }
+    }
+  }
+  float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+  for (int c = 0; c < 128; c += 8) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) mq[q] = fmax3(mq[q], x[c + 2 * q], x[c + 2 * q + 1]);
+  }
+  float mx = fmaxf(fmax3(mq[0], mq[1], mq[2]), mq[3]);
+  if (!prescaled) mx *= p.scale_log2;                // -inf stays -inf (scale > 0)
+  const float m_new = fmaxf(m, mx);
+  float alpha = 1.f;
+  if (m == -INFINITY) {
+    m = m_new;                                       // nothing accumulated yet
+  } else if (m_new > m + kRescaleThreshold) {
+    alpha = ex2_approx(m - m_new);
+    m = m_new;
+  }
+  // pass 2: p = 2^(x * sc - m) (packed FMA), row sum in four packed partial sums
+  const float neg_m = (m == -INFINITY) ? 0.f : -m;
+  const float sc = prescaled ? 1.f : p.scale_log2;
+  float sq[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  if (kEmuPer16 > 0 && !prescaled && !need_mask) {
+#pragma unroll
+    for (int c = 0; c < 128; c += 2) {
+      fma2_bc(x[c], x[c + 1], x[c], x[c + 1], sc, neg_m);
+      if ((c & 15) < kEmuPer16) {
+        exp2_poly2(x[c], x[c + 1]);
+      } else {
+        x[c] = ex2_approx(x[c]);
+        x[c + 1] = ex2_approx(x[c + 1]);
+      }
+      const int q = (c >> 1) & 3;
+      add2(sq[2 * q], sq[2 * q + 1], x[c], x[c + 1]);
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < 128; c += 2) {
+      fma2_bc(x[c], x[c + 1], x[c], x[c + 1], sc, neg_m);
+      x[c] = ex2_approx(x[c]);
+      x[c + 1] = ex2_approx(x[c + 1]);
+      const int q = (c >> 1) & 3;
+      add2(sq[2 * q], sq[2 * q + 1], x[c], x[c + 1]);
+    }
+  }
+  const float sum = ((sq[0] + sq[1]) + (sq[2] + sq[3])) + ((sq[4] + sq[5]) + (sq[6] + sq[7]));
+  l = l * alpha + sum;
+  return alpha;
+}
+
+// Normalised output row (DV values) to global memory; 16-byte stores.
+template <typename T, int DV>
+__device__ __forceinline__ void store_row(const AttnParams &p, const TileInfo &ti, int32_t row,
+                                          const float (&o)[DV], float inv) {
+  T *dst = reinterpret_cast<T *>(p.out) + (int64_t)ti.b * p.o_sb + (int64_t)ti.h * p.o_sh +
+           (int64_t)(p.varlen ? ti.qrow + (row - ti.q0) : row) * p.o_si;
+  if constexpr (sizeof(T) == 2) {
+#pragma unroll
+    for (int c = 0; c < DV; c += 8) {
+      uint4 v;
+      v.x = pack_bf16x2(o[c + 0] * inv, o[c + 1] * inv);
+      v.y = pack_bf16x2(o[c + 2] * inv, o[c + 3] * inv);
+      v.z = pack_bf16x2(o[c + 4] * inv, o[c + 5] * inv);
+      v.w = pack_bf16x2(o[c + 6] * inv, o[c + 7] * inv);
+      *reinterpret_cast<uint4 *>(dst + c) = v;
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < DV; c += 4) {
+      float4 v = make_float4(o[c] * inv, o[c + 1] * inv, o[c + 2] * inv, o[c + 3] * inv);
+      *reinterpret_cast<float4 *>(dst + c) = v;
+    }
+  }
+}
+
+template <typename T, int DV>
+__device__ __forceinline__ void store_zero_row(const AttnParams &p, const TileInfo &ti,
+                                               int32_t row) {
+  float z[DV];
+#pragma unroll
+  for (int c = 0; c < DV; ++c) z[c] = 0.f;
+  store_row<T, DV>(p, ti, row, z, 0.f);
+}
+
+// Load DV fp32 columns of this thread's TMEM lane starting at `taddr`.
+template <int DV>
+__device__ __forceinline__ void tmem_load_row(uint32_t taddr, float (&o)[DV]) {
+#pragma unroll
+  for (int c0 = 0; c0 < DV; c0 += 32) {
+    uint32_t oc[32];
+    tmem_ld_x32(taddr + c0, oc);
+#pragma unroll
+    for (int c = 0; c < 32; ++c) o[c0 + c] = __uint_as_float(oc[c]);
+  }
+}
+
+// O row *= alpha in TMEM (DV columns).
+template <int DV>
+__device__ __forceinline__ void tmem_scale_row(uint32_t taddr, float alpha) {
+#pragma unroll
+  for (int c0 = 0; c0 < DV; c0 += 32) {
+    uint32_t o[32];
+    tmem_ld_x32(taddr + c0, o);
+#pragma unroll
+    for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+    tmem_st_x32(taddr + c0, o);
+  }
+}
+
+// P (128 values) into TMEM over the score columns: bf16 pairs (64 columns),
+// or fp32 bits read by the TF32 MMA (128 columns).
+template <bool kTF32>
+__device__ __forceinline__ void tmem_store_p(uint32_t taddr, const float (&x)[128]) {
+  uint32_t pk[64];
+  if constexpr (!kTF32) {
+#pragma unroll
+    for (int c = 0; c < 64; ++c) pk[c] = pack_bf16x2(x[2 * c], x[2 * c + 1]);
+    tmem_st_x64(taddr, pk);
+  } else {
+#pragma unroll
+    for (int c = 0; c < 64; ++c) pk[c] = __float_as_uint(x[c]);
+    tmem_st_x64(taddr, pk);
+#pragma unroll
+    for (int c = 0; c < 64; ++c) pk[c] = __float_as_uint(x[64 + c]);
+    tmem_st_x64(taddr + 64, pk);
+  }
+}
+
+}  // namespace wf

@@ -1,4 +1,4 @@
-// Explicit instantiations of the attention kernel (f32, d96).
+// Explicit instantiations of the single-tile attention kernel (f32, d96; TF32 MMA).
 // Split across files so the kernels compile in parallel.
 #include "attn_kernel.cuh"
 

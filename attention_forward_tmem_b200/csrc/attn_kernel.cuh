@@ -1,38 +1,29 @@
-// attn_kernel.cuh -- flash-style attention forward for sm_100a.
+// attn_kernel.cuh -- single-tile attention forward for sm_100a (used where
+// two query tiles do not fit in shared memory: the fp32 / TF32 path).
 //
 // Computes, per query row i of head h (kv head g = h / (Hq / Hkv)):
 //     out[i] = sum_j softmax_j(qkScale * (q_i . k_j + qRope_i . kRope_j) + mask_ij) v_j
-// which is the operation of "Core 注意力" (WorldFoundry docs, section
-// "选择最窄的入口": PyTorch SDPA contract with GQA) and of "MLA Prefill" (CANN
-// ATB docs, parameter table: Q/QRope/K/kRope/V, qSeqLen/kvSeqLen, qkScale,
-// maskType).
+// the operation of "Core 注意力" (WorldFoundry docs, section "选择最窄的入口":
+// PyTorch SDPA contract with GQA) and of "MLA Prefill" (CANN ATB docs,
+// parameter table).
 //
-// Design (one CTA per SM, persistent over a longest-first tile list):
-//   warp 4      TMA producer: Q tile once per work tile, then K and V tiles
-//               through a STAGES-deep mbarrier ring (128-byte swizzle).
+// One CTA per SM, persistent over 128-row work units, 192 threads:
+//   warp 4      TMA producer: Q once per unit, then K and V tiles through a
+//               STAGES-deep mbarrier ring (128-byte swizzle).
 //   warp 5      tcgen05 issuer (one thread): S = Q K^T into one of two TMEM
-//               S buffers, then O += P V with P read from TMEM (A operand) and
-//               V from shared memory (MN-major B operand).  S for tile j+1 is
-//               issued before PV for tile j, so the tensor core works on the
-//               next scores while the softmax runs.
-//   warps 0-3   one thread per query row: tcgen05.ld of the score row, scale,
-//               mask (causal / length / explicit), online softmax in the log2
-//               domain with a lazy rescale (the running max is only moved when
-//               it grows by more than 2^8, which is exact after the final
-//               division), P written back over S as bf16 (tf32 for fp32
-//               inputs), O rescaled in TMEM when needed; finally O / l is
-//               stored to global memory.
-//
+//               S buffers, then O += P V with P read from TMEM.  S for tile
+//               j+1 is issued before PV for tile j, so the tensor core works
+//               on the next scores while the softmax runs.
+//   warps 0-3   one thread per query row: softmax_row() on the score row, P
+//               written back over S, O rescaled in TMEM when the running max
+//               moved, finally O / l stored.
 // TMEM columns: S0 [0,128), S1 [128,256), O [256, 256+DV); 512 allocated.
-// Every mbarrier wait is bounded: on expiry the CTA records WF_ERR_TIMEOUT in
-// the device status word, every role leaves its loop, in-flight copies and
-// MMAs are drained (again with a bound) and TMEM is freed.
+// Every mbarrier wait is bounded (see attn_common.cuh).
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
 
-#include "attn_params.h"
-#include "sm100_ptx.cuh"
+#include "attn_common.cuh"
 
 namespace wf {
 
@@ -45,7 +36,11 @@ struct AttnCfg {
   static constexpr int kQAtoms = (DQK + kAtomE - 1) / kAtomE;
   static constexpr int kRAtoms = DROPE / kAtomE;
   static constexpr int kQKAtoms = kQAtoms + kRAtoms;
-  static constexpr int kVAtoms = (DV + kAtomE - 1) / kAtomE;
+  // bf16: V tile [128 keys][DV] used MN-major, DV split into 128-byte atoms.
+  // TF32 (MN-major B not available): V^T tile [DV rows][128 keys] used
+  // K-major, the keys split into 128-byte atoms.
+  static constexpr bool kVKMajor = kTF32;
+  static constexpr int kVAtoms = kVKMajor ? kBlockN / kAtomE : (DV + kAtomE - 1) / kAtomE;
   static constexpr int kAtomBytes = 128 * 128;         // 128 rows x 128 bytes
   static constexpr int kQBytes = kQKAtoms * kAtomBytes;
   static constexpr int kKBytes = kQKAtoms * kAtomBytes;
@@ -67,13 +62,13 @@ struct AttnCfg {
   static constexpr uint32_t kIdescS = instr_desc(kFmt, kBlockM, kBlockN, 0);
   // PV runs over whole 128-byte V atoms (zero-filled past DV by the TMA), so
   // its N never ends inside a swizzle atom.
-  static constexpr int kNPV = kVAtoms * kAtomE;
-  static constexpr uint32_t kIdescPV = instr_desc(kFmt, kBlockM, kNPV, 1);
+  static constexpr int kNPV = kVKMajor ? DV : kVAtoms * kAtomE;
+  static constexpr uint32_t kIdescPV = instr_desc(kFmt, kBlockM, kNPV, kVKMajor ? 0 : 1);
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kOCol = 256;
   static_assert(kStages >= 1, "tile does not fit in shared memory");
   static_assert(DQK % kKStep == 0 && DV % 32 == 0 && DROPE % kAtomE == 0, "head dims");
-  static_assert(DV <= 128 && DV >= 32 && kNPV <= 128, "DV");
+  static_assert(DV <= 128 && DV >= 32 && kNPV <= 128 && kNPV % 16 == 0, "DV");
 };
 
 struct AttnCtrl {
@@ -84,90 +79,7 @@ struct AttnCtrl {
   volatile int32_t abort;
 };
 
-struct TileInfo {
-  int32_t b, h, hk, q0, lq, lk, qrow, krow, n_kv, off, tma_b;
-};
-
-__device__ __forceinline__ TileInfo tile_info(const AttnParams &p, int32_t t) {
-  TileInfo ti;
-  if (!p.varlen) {
-    const int32_t bh = p.batch * p.hq;
-    const int32_t qt = p.nqt_dense - 1 - t / bh;     // longest causal rows first
-    const int32_t r = t % bh;
-    ti.b = r / p.hq;
-    ti.h = r % p.hq;
-    ti.q0 = qt * kBlockM;
-    ti.lq = p.lq;
-    ti.lk = p.lk;
-    ti.qrow = ti.q0;
-    ti.krow = 0;
-    ti.tma_b = ti.b;
-  } else {
-    const int32_t e = t / p.hq;
-    ti.h = t % p.hq;
-    const int32_t *ent = p.ws + p.sl.entries + 2 * e;
-    ti.b = __ldg(ent);
-    const int32_t qt = __ldg(ent + 1);
-    const int32_t cq = __ldg(p.ws + p.sl.cu_q + ti.b), ck = __ldg(p.ws + p.sl.cu_k + ti.b);
-    ti.lq = __ldg(p.ws + p.sl.cu_q + ti.b + 1) - cq;
-    ti.lk = __ldg(p.ws + p.sl.cu_k + ti.b + 1) - ck;
-    ti.q0 = qt * kBlockM;
-    ti.qrow = cq + ti.q0;
-    ti.krow = ck;
-    ti.tma_b = 0;
-  }
-  ti.hk = ti.h / p.group;
-  ti.off = ti.lk - ti.lq;
-  int32_t kend = ti.lk;
-  if (p.mask_kind == kMaskCausal) {
-    const int32_t last = min(ti.q0 + kBlockM, ti.lq);   // one past the last valid row
-    kend = min(kend, last + ti.off);
-  }
-  ti.n_kv = kend > 0 ? (kend + kBlockN - 1) / kBlockN : 0;
-  return ti;
-}
-
-__device__ __forceinline__ int32_t num_tiles(const AttnParams &p) {
-  if (!p.varlen) return p.n_tiles_dense;
-  return __ldg(p.ws) * p.hq;
-}
-
-// Bounded wait.  Returns false (and raises the CTA abort flag) on expiry, or
-// if another role already aborted.
-__device__ __forceinline__ bool bwait(uint64_t *bar, uint32_t parity, AttnCtrl *ctl,
-                                      const AttnParams &p) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const long long t0 = clock64();
-  while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (ctl->abort) return false;
-    if (clock64() - t0 > p.timeout_cycles) {
-      ctl->abort = 1;
-      atomicCAS(p.status, 0, kDevTimeout);
-      return false;
-    }
-  }
-}
-
-// Wait used while draining after an abort: ignores the abort flag, still bounded.
-__device__ __forceinline__ bool drain_wait(uint64_t *bar, uint32_t parity, const AttnParams &p) {
-  const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > p.timeout_cycles) {
-      atomicCAS(p.status, 0, kDevTimeout);
-      return false;
-    }
-  }
-  return true;
-}
-
 // ------------------------------------------------------------------ producer
-// Last fill index the producer issued per barrier (-1: none), for the drain.
-struct ProducerLog {
-  int32_t q_last;
-  int32_t k_last[3], v_last[3];
-};
-
 template <typename Cfg>
 __device__ void producer_role(const AttnParams &p, uint8_t *smem, AttnCtrl *ctl,
                               ProducerLog &log) {
@@ -178,17 +90,17 @@ __device__ void producer_role(const AttnParams &p, uint8_t *smem, AttnCtrl *ctl,
     tma_prefetch_map(&p.tm_qr);
     tma_prefetch_map(&p.tm_kr);
   }
-  const int32_t n_tiles = num_tiles(p);
+  const int32_t n_units = num_units(p);
   uint32_t g = 0, u = 0;
   int32_t *k_last = log.k_last, *v_last = log.v_last;
   log.q_last = -1;
   for (int i = 0; i < 3; ++i) k_last[i] = v_last[i] = -1;
   bool ok = true;
   bool starve = (p.debug_flags & kDebugStarveFirstK) != 0;
-  for (int32_t t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
-    const TileInfo ti = tile_info(p, t);
+  for (int32_t t = blockIdx.x; t < n_units && ok; t += gridDim.x) {
+    const TileInfo ti = tile_info(p, t, 0);
     if (ti.n_kv == 0) continue;
-    if (!(ok = bwait(&ctl->q_empty, (u + 1) & 1, ctl, p))) break;
+    if (!(ok = bwait(&ctl->q_empty, (u + 1) & 1, &ctl->abort, p))) break;
     mbar_arrive_expect_tx(&ctl->q_full, Cfg::kQBytes);
     log.q_last = static_cast<int32_t>(u);
 #pragma unroll
@@ -202,7 +114,7 @@ __device__ void producer_role(const AttnParams &p, uint8_t *smem, AttnCtrl *ctl,
     for (int32_t j = 0; j < ti.n_kv; ++j) {
       const uint32_t gg = g + j, st = gg % Cfg::kStages, n = gg / Cfg::kStages;
       const int32_t krow = ti.krow + j * kBlockN;
-      if (!(ok = bwait(&ctl->k_empty[st], (n + 1) & 1, ctl, p))) break;
+      if (!(ok = bwait(&ctl->k_empty[st], (n + 1) & 1, &ctl->abort, p))) break;
       if (starve) {
         starve = false;     // debug: this K tile is never loaded, its consumer times out
       } else {
@@ -218,13 +130,18 @@ __device__ void producer_role(const AttnParams &p, uint8_t *smem, AttnCtrl *ctl,
                       a * Cfg::kAtomE, krow, ti.hk, ti.tma_b);
         k_last[st] = static_cast<int32_t>(n);
       }
-      if (!(ok = bwait(&ctl->v_empty[st], (n + 1) & 1, ctl, p))) break;
+      if (!(ok = bwait(&ctl->v_empty[st], (n + 1) & 1, &ctl->abort, p))) break;
       uint8_t *vdst = smem + Cfg::kVOff + st * Cfg::kVBytes;
       mbar_arrive_expect_tx(&ctl->v_full[st], Cfg::kVBytes);
 #pragma unroll
-      for (int a = 0; a < Cfg::kVAtoms; ++a)
-        tma_load_4d(vdst + a * Cfg::kAtomBytes, &p.tm_v, &ctl->v_full[st], a * Cfg::kAtomE, krow,
-                    ti.hk, ti.tma_b);
+      for (int a = 0; a < Cfg::kVAtoms; ++a) {
+        if constexpr (Cfg::kVKMajor)   // V^T: (keys, DV rows) box at key offset a*kAtomE
+          tma_load_4d(vdst + a * Cfg::kAtomBytes, &p.tm_v, &ctl->v_full[st], krow + a * Cfg::kAtomE,
+                      0, ti.hk, ti.tma_b);
+        else
+          tma_load_4d(vdst + a * Cfg::kAtomBytes, &p.tm_v, &ctl->v_full[st], a * Cfg::kAtomE, krow,
+                      ti.hk, ti.tma_b);
+      }
       v_last[st] = static_cast<int32_t>(n);
     }
     if (!ok) break;
@@ -236,13 +153,14 @@ __device__ void producer_role(const AttnParams &p, uint8_t *smem, AttnCtrl *ctl,
 // Wait (bounded) for every copy the producer started, so that no TMA write
 // can land after the CTA has released its shared memory.  Run after all roles
 // finished; in a normal run every one of these phases is already complete.
-template <typename Cfg>
-__device__ void producer_drain(const AttnParams &p, AttnCtrl *ctl, const ProducerLog &log) {
+template <typename Ctrl>
+__device__ void producer_drain(const AttnParams &p, Ctrl *ctl, const ProducerLog &log,
+                               int k_stages, int v_stages) {
   if (log.q_last >= 0) drain_wait(&ctl->q_full, log.q_last & 1, p);
-  for (int s = 0; s < Cfg::kStages; ++s) {
+  for (int s = 0; s < k_stages; ++s)
     if (log.k_last[s] >= 0) drain_wait(&ctl->k_full[s], log.k_last[s] & 1, p);
+  for (int s = 0; s < v_stages; ++s)
     if (log.v_last[s] >= 0) drain_wait(&ctl->v_full[s], log.v_last[s] & 1, p);
-  }
 }
 
 // ----------------------------------------------------------------------- MMA
@@ -251,15 +169,16 @@ __device__ __forceinline__ void issue_pv(const AttnParams &p, uint8_t *smem, Att
                                          uint32_t tmem, uint32_t gg, bool first, uint32_t u,
                                          bool &ok) {
   const uint32_t st = gg % Cfg::kStages, sb = gg & 1;
-  if (first && !(ok = bwait(&ctl->o_empty, (u + 1) & 1, ctl, p))) return;
-  if (!(ok = bwait(&ctl->p_full[sb], (gg >> 1) & 1, ctl, p))) return;
-  if (!(ok = bwait(&ctl->v_full[st], (gg / Cfg::kStages) & 1, ctl, p))) return;
+  if (first && !(ok = bwait(&ctl->o_empty, (u + 1) & 1, &ctl->abort, p))) return;
+  if (!(ok = bwait(&ctl->p_full[sb], (gg >> 1) & 1, &ctl->abort, p))) return;
+  if (!(ok = bwait(&ctl->v_full[st], (gg / Cfg::kStages) & 1, &ctl->abort, p))) return;
   tc_fence_after();
   const uint32_t vbase = smem_u32(smem + Cfg::kVOff + st * Cfg::kVBytes);
 #pragma unroll
   for (int ks = 0; ks < Cfg::kPVKSteps; ++ks) {
     const uint64_t bdesc =
-        smem_desc_sw128(vbase + ks * Cfg::kKStep * 128, Cfg::kAtomBytes, 1024);
+        Cfg::kVKMajor ? smem_desc_sw128(vbase + (ks / 4) * Cfg::kAtomBytes + (ks % 4) * 32, 16, 1024)
+                      : smem_desc_sw128(vbase + ks * Cfg::kKStep * 128, Cfg::kAtomBytes, 1024);
     const uint32_t a_tmem = tmem + sb * 128 + ks * 8;
     if constexpr (Cfg::kTF32)
       mma_tf32_ts(tmem + Cfg::kOCol, a_tmem, bdesc, Cfg::kIdescPV, (!first || ks > 0) ? 1u : 0u);
@@ -272,20 +191,20 @@ __device__ __forceinline__ void issue_pv(const AttnParams &p, uint8_t *smem, Att
 
 template <typename Cfg>
 __device__ void mma_role(const AttnParams &p, uint8_t *smem, AttnCtrl *ctl, uint32_t tmem) {
-  const int32_t n_tiles = num_tiles(p);
+  const int32_t n_units = num_units(p);
   const uint32_t qbase = smem_u32(smem);
   uint32_t g = 0, u = 0;
   bool ok = true;
-  for (int32_t t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
-    const TileInfo ti = tile_info(p, t);
+  for (int32_t t = blockIdx.x; t < n_units && ok; t += gridDim.x) {
+    const TileInfo ti = tile_info(p, t, 0);
     if (ti.n_kv == 0) continue;
-    if (!(ok = bwait(&ctl->q_full, u & 1, ctl, p))) break;
+    if (!(ok = bwait(&ctl->q_full, u & 1, &ctl->abort, p))) break;
     tc_fence_after();
     for (int32_t j = 0; j < ti.n_kv; ++j) {
       const uint32_t gg = g + j, st = gg % Cfg::kStages, sb = gg & 1;
-      if (!(ok = bwait(&ctl->k_full[st], (gg / Cfg::kStages) & 1, ctl, p))) break;
+      if (!(ok = bwait(&ctl->k_full[st], (gg / Cfg::kStages) & 1, &ctl->abort, p))) break;
       // S buffer sb was last read (as P) by PV[gg-2]
-      if (gg >= 2 && !(ok = bwait(&ctl->pv_done[sb], ((gg - 2) >> 1) & 1, ctl, p))) break;
+      if (gg >= 2 && !(ok = bwait(&ctl->pv_done[sb], ((gg - 2) >> 1) & 1, &ctl->abort, p))) break;
       tc_fence_after();
       const uint32_t kbase = smem_u32(smem + Cfg::kKOff + st * Cfg::kKBytes);
 #pragma unroll
@@ -322,151 +241,39 @@ __device__ void mma_role(const AttnParams &p, uint8_t *smem, AttnCtrl *ctl, uint
 
 // ------------------------------------------------------------------- softmax
 template <typename T, typename Cfg, int DV>
-__device__ __forceinline__ void store_row(const AttnParams &p, const TileInfo &ti, int32_t row,
-                                          const float (&o)[DV], float inv) {
-  T *dst = reinterpret_cast<T *>(p.out) + (int64_t)ti.b * p.o_sb + (int64_t)ti.h * p.o_sh +
-           (int64_t)(p.varlen ? ti.qrow + (row - ti.q0) : row) * p.o_si;
-  if constexpr (sizeof(T) == 2) {
-#pragma unroll
-    for (int c = 0; c < DV; c += 8) {
-      uint4 v;
-      v.x = pack_bf16x2(o[c + 0] * inv, o[c + 1] * inv);
-      v.y = pack_bf16x2(o[c + 2] * inv, o[c + 3] * inv);
-      v.z = pack_bf16x2(o[c + 4] * inv, o[c + 5] * inv);
-      v.w = pack_bf16x2(o[c + 6] * inv, o[c + 7] * inv);
-      *reinterpret_cast<uint4 *>(dst + c) = v;
-    }
-  } else {
-#pragma unroll
-    for (int c = 0; c < DV; c += 4) {
-      float4 v = make_float4(o[c] * inv, o[c + 1] * inv, o[c + 2] * inv, o[c + 3] * inv);
-      *reinterpret_cast<float4 *>(dst + c) = v;
-    }
-  }
-}
-
-template <typename T, typename Cfg, int DV>
 __device__ void softmax_role(const AttnParams &p, AttnCtrl *ctl, uint32_t tmem) {
   const int32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int32_t r = threadIdx.x;                       // row within the tile = TMEM lane
   const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-  const int32_t n_tiles = num_tiles(p);
-  const bool causal = p.mask_kind == kMaskCausal;
-  const bool explicit_mask = p.mask_kind == kMaskKeep || p.mask_kind == kMaskAdd;
-  constexpr float kLog2e = 1.4426950408889634f;
-  constexpr float kRescaleThreshold = 8.0f;            // log2 units
+  const int32_t n_units = num_units(p);
   uint32_t g = 0;
   bool ok = true;
-  for (int32_t t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
-    const TileInfo ti = tile_info(p, t);
+  for (int32_t t = blockIdx.x; t < n_units && ok; t += gridDim.x) {
+    const TileInfo ti = tile_info(p, t, 0);
     const int32_t row = ti.q0 + r;
     const bool row_valid = row < ti.lq;
     if (ti.n_kv == 0) {
-      if (row_valid) {
-        float z[DV];
-#pragma unroll
-        for (int c = 0; c < DV; ++c) z[c] = 0.f;
-        store_row<T, Cfg, DV>(p, ti, row, z, 0.f);
-      }
+      if (row_valid) store_zero_row<T, DV>(p, ti, row);
       continue;
     }
     float m = -INFINITY, l = 0.f;
     for (int32_t j = 0; j < ti.n_kv; ++j) {
       const uint32_t gg = g + j, sb = gg & 1;
-      if (!(ok = bwait(&ctl->s_full[sb], (gg >> 1) & 1, ctl, p))) break;
+      if (!(ok = bwait(&ctl->s_full[sb], (gg >> 1) & 1, &ctl->abort, p))) break;
       tc_fence_after();
       uint32_t sr[128];
       tmem_ld_x128(tmem + lane_base + sb * 128, sr);
       float x[128];
-      const int32_t k0 = j * kBlockN;
-      int32_t lim = ti.lk - 1 - k0;                    // last visible column of this row
-      if (causal) lim = min(lim, row + ti.off - k0);
-      const bool need_mask =
-          explicit_mask || (k0 + kBlockN > ti.lk) || (causal && (k0 + kBlockN - 1 > ti.q0 + ti.off));
-      if (!explicit_mask) {
-        if (need_mask) {
-#pragma unroll
-          for (int c = 0; c < 128; ++c)
-            x[c] = (c <= lim) ? __uint_as_float(sr[c]) * p.scale_log2 : -INFINITY;
-        } else {
-#pragma unroll
-          for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(sr[c]) * p.scale_log2;
-        }
-      } else {
-        const int64_t mrow = (int64_t)ti.b * p.m_sb + (int64_t)ti.h * p.m_sh + (int64_t)row * p.m_si;
-        if (p.mask_kind == kMaskKeep) {
-          const uint8_t *mp = reinterpret_cast<const uint8_t *>(p.mask) + mrow;
-#pragma unroll
-          for (int c = 0; c < 128; ++c) {
-            const bool keep = row_valid && c <= lim && mp[(int64_t)(k0 + c) * p.m_sj] != 0;
-            x[c] = keep ? __uint_as_float(sr[c]) * p.scale_log2 : -INFINITY;
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < 128; ++c) {
-            float add = 0.f;
-            const bool in = row_valid && c <= lim;
-            if (in) {
-              const int64_t idx = mrow + (int64_t)(k0 + c) * p.m_sj;
-              add = p.mask_dtype == kMaskF32
-                        ? reinterpret_cast<const float *>(p.mask)[idx]
-                        : __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(p.mask)[idx]);
-            }
-            x[c] = in ? fmaf(add, kLog2e, __uint_as_float(sr[c]) * p.scale_log2) : -INFINITY;
-          }
-        }
-      }
-      float mx = x[0];
-#pragma unroll
-      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, x[c]);
-      const float m_new = fmaxf(m, mx);
-      float alpha = 1.f;
-      bool rescale = false;
-      if (m == -INFINITY) {
-        m = m_new;                                     // nothing accumulated yet
-      } else if (m_new > m + kRescaleThreshold) {
-        alpha = ex2_approx(m - m_new);
-        m = m_new;
-        rescale = true;
-      }
-      const float m_use = (m == -INFINITY) ? 0.f : m;
-      float sum = 0.f;
-#pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        x[c] = ex2_approx(x[c] - m_use);
-        sum += x[c];
-      }
-      l = l * alpha + sum;
-      // P over S (same TMEM columns): bf16 pairs, or fp32 bits read as tf32.
-      if constexpr (!Cfg::kTF32) {
-        uint32_t pk[64];
-#pragma unroll
-        for (int c = 0; c < 64; ++c) pk[c] = pack_bf16x2(x[2 * c], x[2 * c + 1]);
-        tmem_st_x64(tmem + lane_base + sb * 128, pk);
-      } else {
-        uint32_t pk[64];
-#pragma unroll
-        for (int c = 0; c < 64; ++c) pk[c] = __float_as_uint(x[c]);
-        tmem_st_x64(tmem + lane_base + sb * 128, pk);
-#pragma unroll
-        for (int c = 0; c < 64; ++c) pk[c] = __float_as_uint(x[64 + c]);
-        tmem_st_x64(tmem + lane_base + sb * 128 + 64, pk);
-      }
-      if (j > 0 && __any_sync(0xffffffffu, rescale)) {
+      const float alpha = softmax_row<0>(p, ti, row, j * kBlockN, sr, x, m, l);
+      tmem_store_p<Cfg::kTF32>(tmem + lane_base + sb * 128, x);
+      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
         // O holds the sum up to tile j-1 once PV[gg-1] is done.
-        if (!(ok = bwait(&ctl->pv_done[(gg - 1) & 1], ((gg - 1) >> 1) & 1, ctl, p))) {
+        if (!(ok = bwait(&ctl->pv_done[(gg - 1) & 1], ((gg - 1) >> 1) & 1, &ctl->abort, p))) {
           tmem_st_wait();
           break;
         }
         tc_fence_after();
-#pragma unroll
-        for (int c0 = 0; c0 < DV; c0 += 32) {
-          uint32_t o[32];
-          tmem_ld_x32(tmem + lane_base + Cfg::kOCol + c0, o);
-#pragma unroll
-          for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-          tmem_st_x32(tmem + lane_base + Cfg::kOCol + c0, o);
-        }
+        tmem_scale_row<DV>(tmem + lane_base + Cfg::kOCol, alpha);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -477,20 +284,14 @@ __device__ void softmax_role(const AttnParams &p, AttnCtrl *ctl, uint32_t tmem) 
     g += ti.n_kv;
     // Epilogue: O is final once the last PV of this tile is done.
     const uint32_t gl = g - 1;
-    if (!(ok = bwait(&ctl->pv_done[gl & 1], (gl >> 1) & 1, ctl, p))) break;
+    if (!(ok = bwait(&ctl->pv_done[gl & 1], (gl >> 1) & 1, &ctl->abort, p))) break;
     tc_fence_after();
     float o[DV];
-#pragma unroll
-    for (int c0 = 0; c0 < DV; c0 += 32) {
-      uint32_t oc[32];
-      tmem_ld_x32(tmem + lane_base + Cfg::kOCol + c0, oc);
-#pragma unroll
-      for (int c = 0; c < 32; ++c) o[c0 + c] = __uint_as_float(oc[c]);
-    }
+    tmem_load_row<DV>(tmem + lane_base + Cfg::kOCol, o);
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(&ctl->o_empty);
-    if (row_valid) store_row<T, Cfg, DV>(p, ti, row, o, l > 0.f ? 1.f / l : 0.f);
+    if (row_valid) store_row<T, DV>(p, ti, row, o, l > 0.f ? 1.f / l : 0.f);
   }
 }
 
@@ -548,7 +349,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     tc_fence_after();
     tmem_dealloc(tmem, Cfg::kTmemCols);
   } else if (warp == 4 && (threadIdx.x & 31) == 0) {
-    producer_drain<Cfg>(p, ctl, plog);
+    producer_drain(p, ctl, plog, Cfg::kStages, Cfg::kStages);
   }
 }
 

@@ -24,15 +24,17 @@ constexpr uint32_t kDebugStarveFirstK = 1u;   // producer never loads the first 
 // Varlen schedule workspace (int32 words):
 //   [0] number of (sequence, q-tile) entries E, [1] length-check flag,
 //   [cu_q .. cu_q+B] and [cu_k .. cu_k+B] prefix sums of the lengths,
-//   [cu_t .. cu_t+B] prefix sums of q tiles per sequence,
-//   [entries ..] E pairs (sequence, q tile), longest KV range first.
+//   [cu_t .. cu_t+B] prefix sums of work units per sequence,
+//   [entries ..] E pairs (sequence, unit), longest KV range first.
+// A work unit is `unit_rows` consecutive query rows of one sequence.
 struct SchedLayout {
   int32_t cu_q, cu_k, cu_t, entries, capacity;   // offsets in words; capacity in entries
   int64_t words;
 };
 
 struct alignas(64) AttnParams {
-  CUtensorMap tm_q, tm_k, tm_v, tm_qr, tm_kr;   // 4-d maps (D, rows, heads, batch)
+  CUtensorMap tm_q, tm_k, tm_v, tm_qr, tm_kr;   // 4-d maps (D, rows, heads, batch);
+                                                 // fp32: tm_v maps V^T (rows, D, heads, batch)
   void *out;
   int64_t o_sb, o_sh, o_si;                      // element strides of out (batch, head, row)
   const void *mask;
@@ -41,7 +43,8 @@ struct alignas(64) AttnParams {
   int32_t batch, hq, hkv, group;
   int32_t lq, lk;                                // dense lengths
   int32_t varlen;
-  int32_t n_tiles_dense, nqt_dense;
+  int32_t unit_rows;                             // query rows per work unit (128 or 256)
+  int32_t n_units_dense, units_per_bh;           // dense: total units, units per (b, h)
   const int32_t *ws;                             // varlen schedule (device)
   SchedLayout sl;
   float scale_log2;                              // qkScale * log2(e)
@@ -52,12 +55,22 @@ struct alignas(64) AttnParams {
 
 using AttnLaunchFn = cudaError_t (*)(const AttnParams &, int grid, cudaStream_t);
 
-// Returns the launcher for (dtype 0 = f32 / 1 = bf16, dqk, drope, dv), or nullptr.
-AttnLaunchFn find_attn_kernel(int dtype, int dqk, int drope, int dv);
+struct AttnKernel {
+  AttnLaunchFn launch;
+  int32_t unit_rows;     // query rows per work unit of this kernel
+};
+
+// Kernel for (dtype 0 = f32 / 1 = bf16, dqk, drope, dv); launch == nullptr if none.
+AttnKernel find_attn_kernel(int dtype, int dqk, int drope, int dv);
+
+// V [rows, heads, batch] x d (element strides) -> V^T [batch][heads][d][ld] (fp32).
+cudaError_t launch_transpose_v(const float *v, int64_t s_row, int64_t s_head, int64_t s_batch,
+                               int32_t rows, int32_t heads, int32_t batch, int32_t d, float *vt,
+                               int64_t ld, cudaStream_t stream);
 
 cudaError_t launch_sched_prep(const int32_t *q_len, const int32_t *k_len, int32_t batch,
                               int64_t n_q_tokens, int64_t n_k_tokens, int32_t causal,
-                              int32_t *ws, const SchedLayout &sl, int32_t *status,
-                              cudaStream_t stream);
+                              int32_t unit_rows, int32_t *ws, const SchedLayout &sl,
+                              int32_t *status, cudaStream_t stream);
 
 }  // namespace wf

@@ -1,0 +1,391 @@
+// attn_pingpong.cuh -- two-tile ("ping-pong") attention forward for sm_100a,
+// bf16 inputs.
+//
+// Same operation as attn_kernel.cuh ("Core 注意力" section "选择最窄的入口";
+// "MLA Prefill" parameter table).  A CTA owns a 256-row work unit: two
+// 128-row query tiles A and B of one (sequence, head) that share every K and
+// V tile.  Each tile has its own TMEM score buffer, its own TMEM output
+// accumulator and its own softmax warpgroup; the single MMA thread issues
+//     PV_A(j-1), S_A(j), PV_B(j-1), S_B(j)
+// so the tensor core computes one tile's products while the other tile's
+// softmax runs.  S_A(j) overwrites the columns PV_A(j-1) reads P from; it is
+// issued after PV_A(j-1) by the same thread, and tcgen05 MMAs from one thread
+// execute in issue order.  The same ordering also means that when a softmax
+// warpgroup sees S_s(j) complete, PV_s(j-1) has completed, so it can rescale
+// O_s in TMEM without a further wait.
+//
+// Warps: 0-3 softmax of tile A (one thread per row), 4-7 softmax of tile B,
+// 8 TMA producer, 9 MMA issuer, 10-11 idle (they only complete warpgroup 2 so
+// that its register limit can be lowered in favour of the softmax groups).  TMEM: S_A [0,128), S_B [128,256),
+// O_A [256,384), O_B [384,512).  Shared memory: Q_A, Q_B, then K and V rings
+// (separate depths, so the 192-wide MLA tiles still fit).
+#pragma once
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "attn_common.cuh"
+
+namespace wf {
+
+constexpr int kPPThreads = 384;            // 3 warpgroups
+constexpr uint32_t kPPSoftmaxRegs = 192;    // warpgroups 0 and 1
+constexpr uint32_t kPPOtherRegs = 120;       // warpgroup 2: producer, MMA, 2 idle warps
+// launch: 384 threads x 168 registers = 64512 >= 2*128*200 + 128*96 = 63488
+static_assert(2 * 128 * kPPSoftmaxRegs + 128 * kPPOtherRegs <= kPPThreads * 168, "register split");
+
+template <int DQK, int DROPE, int DV>
+struct PPCfg {
+  static constexpr int kAtomE = 64;                       // bf16 elements per 128-byte row
+  static constexpr int kKStep = 16;
+  static constexpr int kQAtoms = (DQK + kAtomE - 1) / kAtomE;
+  static constexpr int kRAtoms = DROPE / kAtomE;
+  static constexpr int kQKAtoms = kQAtoms + kRAtoms;
+  static constexpr int kVAtoms = (DV + kAtomE - 1) / kAtomE;
+  static constexpr int kAtomBytes = 128 * 128;
+  static constexpr int kQTileBytes = kQKAtoms * kAtomBytes;
+  static constexpr int kQBytes = 2 * kQTileBytes;
+  static constexpr int kKBytes = kQKAtoms * kAtomBytes;
+  static constexpr int kVBytes = kVAtoms * kAtomBytes;
+  static constexpr int kBudget = 227 * 1024 - 2048;
+  static constexpr int kEqFit = (kBudget - kQBytes) / (kKBytes + kVBytes);
+  static constexpr bool kTwoOne = kEqFit < 2 && (kBudget - kQBytes - 2 * kKBytes - kVBytes) >= 0;
+  static constexpr int kKStages = kEqFit >= 3 ? 3 : (kEqFit == 2 ? 2 : (kTwoOne ? 2 : 1));
+  static constexpr int kVStages = kEqFit >= 3 ? 3 : (kEqFit == 2 ? 2 : 1);
+  static constexpr int kKOff = kQBytes;
+  static constexpr int kVOff = kKOff + kKStages * kKBytes;
+  static constexpr int kCtrlOff = kVOff + kVStages * kVBytes;
+  static constexpr int kSmemUsed = kCtrlOff + 1024 + 1024;
+  static constexpr int kSmemBytes = kSmemUsed > 120 * 1024 ? kSmemUsed : 120 * 1024;
+  static constexpr int kSKStepsQK = DQK / kKStep;
+  static constexpr int kSKStepsR = DROPE / kKStep;
+  static constexpr int kPVKSteps = kBlockN / kKStep;
+  static constexpr int kNPV = kVAtoms * kAtomE;
+  static constexpr uint32_t kIdescS = instr_desc(1, kBlockM, kBlockN, 0);
+  static constexpr uint32_t kIdescPV = instr_desc(1, kBlockM, kNPV, 1);
+  static constexpr uint32_t kTmemCols = 512;
+  // FMA-pipe exp2 share (of 16 columns): pays off where the QK product is 128
+  // wide; the 192-wide MLA product leaves the softmax enough time as it is.
+  static constexpr int kEmuPer16 = (DQK + DROPE) <= 128 ? 4 : 0;
+  static_assert(kKStages >= 1 && kVStages >= 1 && kSmemUsed <= 227 * 1024, "smem");
+  static_assert(DQK % kKStep == 0 && DV % 32 == 0 && kNPV <= 128, "head dims");
+};
+
+struct PPCtrl {
+  uint64_t q_full, q_empty, drain;
+  uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
+  uint64_t k_full[3], k_empty[3], v_full[3], v_empty[3];
+  uint32_t tmem_base;
+  volatile int32_t abort;
+};
+
+// ------------------------------------------------------------------ producer
+template <typename Cfg>
+__device__ void pp_producer(const AttnParams &p, uint8_t *smem, PPCtrl *ctl, ProducerLog &log) {
+  tma_prefetch_map(&p.tm_q);
+  tma_prefetch_map(&p.tm_k);
+  tma_prefetch_map(&p.tm_v);
+  if (Cfg::kRAtoms) {
+    tma_prefetch_map(&p.tm_qr);
+    tma_prefetch_map(&p.tm_kr);
+  }
+  const int32_t n_units = num_units(p);
+  uint32_t g = 0, u = 0;
+  log.q_last = -1;
+  for (int i = 0; i < 3; ++i) log.k_last[i] = log.v_last[i] = -1;
+  bool ok = true;
+  bool starve = (p.debug_flags & kDebugStarveFirstK) != 0;
+
+  auto load_k = [&](const TileInfo &ti, int32_t j) -> bool {
+    const uint32_t gg = g + j, st = gg % Cfg::kKStages, n = gg / Cfg::kKStages;
+    if (!bwait(&ctl->k_empty[st], (n + 1) & 1, &ctl->abort, p)) return false;
+    if (starve) {                     // debug: never load this K tile
+      starve = false;
+      return true;
+    }
+    const int32_t krow = ti.krow + j * kBlockN;
+    uint8_t *dst = smem + Cfg::kKOff + st * Cfg::kKBytes;
+    mbar_arrive_expect_tx(&ctl->k_full[st], Cfg::kKBytes);
+#pragma unroll
+    for (int a = 0; a < Cfg::kQAtoms; ++a)
+      tma_load_4d(dst + a * Cfg::kAtomBytes, &p.tm_k, &ctl->k_full[st], a * Cfg::kAtomE, krow,
+                  ti.hk, ti.tma_b);
+#pragma unroll
+    for (int a = 0; a < Cfg::kRAtoms; ++a)
+      tma_load_4d(dst + (Cfg::kQAtoms + a) * Cfg::kAtomBytes, &p.tm_kr, &ctl->k_full[st],
+                  a * Cfg::kAtomE, krow, ti.hk, ti.tma_b);
+    log.k_last[st] = static_cast<int32_t>(n);
+    return true;
+  };
+  auto load_v = [&](const TileInfo &ti, int32_t j) -> bool {
+    const uint32_t gg = g + j, st = gg % Cfg::kVStages, n = gg / Cfg::kVStages;
+    if (!bwait(&ctl->v_empty[st], (n + 1) & 1, &ctl->abort, p)) return false;
+    const int32_t krow = ti.krow + j * kBlockN;
+    uint8_t *dst = smem + Cfg::kVOff + st * Cfg::kVBytes;
+    mbar_arrive_expect_tx(&ctl->v_full[st], Cfg::kVBytes);
+#pragma unroll
+    for (int a = 0; a < Cfg::kVAtoms; ++a)
+      tma_load_4d(dst + a * Cfg::kAtomBytes, &p.tm_v, &ctl->v_full[st], a * Cfg::kAtomE, krow,
+                  ti.hk, ti.tma_b);
+    log.v_last[st] = static_cast<int32_t>(n);
+    return true;
+  };
+
+  for (int32_t t = blockIdx.x; t < n_units && ok; t += gridDim.x) {
+    const TileInfo t0 = tile_info(p, t, 0), t1 = tile_info(p, t, 1);
+    const int32_t n_max = max(t0.n_kv, t1.n_kv);
+    if (n_max == 0) continue;
+    if (!(ok = bwait(&ctl->q_empty, (u + 1) & 1, &ctl->abort, p))) break;
+    mbar_arrive_expect_tx(&ctl->q_full, Cfg::kQBytes);
+    log.q_last = static_cast<int32_t>(u);
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      const TileInfo &ts = s ? t1 : t0;
+      uint8_t *qdst = smem + s * Cfg::kQTileBytes;
+#pragma unroll
+      for (int a = 0; a < Cfg::kQAtoms; ++a)
+        tma_load_4d(qdst + a * Cfg::kAtomBytes, &p.tm_q, &ctl->q_full, a * Cfg::kAtomE, ts.qrow,
+                    ts.h, ts.tma_b);
+#pragma unroll
+      for (int a = 0; a < Cfg::kRAtoms; ++a)
+        tma_load_4d(qdst + (Cfg::kQAtoms + a) * Cfg::kAtomBytes, &p.tm_qr, &ctl->q_full,
+                    a * Cfg::kAtomE, ts.qrow, ts.h, ts.tma_b);
+    }
+    // consumption order of the MMA thread: K0, then per j: V(j-1), K(j)...;
+    // keep K one tile ahead of V.
+    if (!(ok = load_k(t0, 0))) break;
+    for (int32_t j = 0; j < n_max && ok; ++j) {
+      if (j + 1 < n_max && !(ok = load_k(t0, j + 1))) break;
+      ok = load_v(t0, j);
+    }
+    if (!ok) break;
+    g += n_max;
+    ++u;
+  }
+}
+
+// ----------------------------------------------------------------------- MMA
+template <typename Cfg>
+__device__ __forceinline__ void pp_issue_s(uint32_t tmem, uint32_t qbase, uint32_t kbase,
+                                           int s) {
+#pragma unroll
+  for (int ks = 0; ks < Cfg::kSKStepsQK + Cfg::kSKStepsR; ++ks) {
+    const int atom = ks < Cfg::kSKStepsQK ? ks / 4 : Cfg::kQAtoms + (ks - Cfg::kSKStepsQK) / 4;
+    const int within = (ks < Cfg::kSKStepsQK ? ks % 4 : (ks - Cfg::kSKStepsQK) % 4) * 32;
+    const uint32_t off = atom * Cfg::kAtomBytes + within;
+    mma_f16_ss(tmem + (s ? 128u : 0u), smem_desc_sw128(qbase + off, 16, 1024),
+               smem_desc_sw128(kbase + off, 16, 1024), Cfg::kIdescS, ks > 0 ? 1u : 0u);
+  }
+}
+
+template <typename Cfg>
+__device__ __forceinline__ void pp_issue_pv(uint32_t tmem, uint32_t vbase, int s, bool accumulate) {
+#pragma unroll
+  for (int ks = 0; ks < Cfg::kPVKSteps; ++ks) {
+    const uint64_t bdesc = smem_desc_sw128(vbase + ks * Cfg::kKStep * 128, Cfg::kAtomBytes, 1024);
+    mma_f16_ts(tmem + (s ? 384u : 256u), tmem + (s ? 128u : 0u) + ks * 8, bdesc, Cfg::kIdescPV,
+               (accumulate || ks > 0) ? 1u : 0u);
+  }
+}
+
+template <typename Cfg>
+__device__ void pp_mma(const AttnParams &p, uint8_t *smem, PPCtrl *ctl, uint32_t tmem) {
+  const int32_t n_units = num_units(p);
+  uint32_t g = 0, u = 0;
+  uint32_t cp[2] = {0, 0};    // PVs issued per tile slot (p_full completions consumed)
+  uint32_t co[2] = {0, 0};    // units in which each tile slot took part (o_empty phases)
+  bool ok = true;
+  const uint32_t qb[2] = {smem_u32(smem), smem_u32(smem + Cfg::kQTileBytes)};
+  auto kbase = [&](uint32_t gg) { return smem_u32(smem + Cfg::kKOff + (gg % Cfg::kKStages) * Cfg::kKBytes); };
+  auto vbase = [&](uint32_t gg) { return smem_u32(smem + Cfg::kVOff + (gg % Cfg::kVStages) * Cfg::kVBytes); };
+  auto wait_k = [&](uint32_t gg) {
+    return bwait(&ctl->k_full[gg % Cfg::kKStages], (gg / Cfg::kKStages) & 1, &ctl->abort, p);
+  };
+  auto wait_v = [&](uint32_t gg) {
+    return bwait(&ctl->v_full[gg % Cfg::kVStages], (gg / Cfg::kVStages) & 1, &ctl->abort, p);
+  };
+  // PV of tile slot s for KV tile (unit-local) jj; returns false on abort.
+  auto do_pv = [&](int s, int32_t jj, int32_t n_s, uint32_t gg) -> bool {
+    if (jj == 0 && !bwait(&ctl->o_empty[s], (co[s] + 1) & 1, &ctl->abort, p)) return false;
+    if (!bwait(&ctl->p_full[s], cp[s] & 1, &ctl->abort, p)) return false;
+    tc_fence_after();
+    pp_issue_pv<Cfg>(tmem, vbase(gg), s, jj > 0);
+    ++cp[s];
+    if (jj == n_s - 1) tc_commit(&ctl->o_full[s]);
+    return true;
+  };
+
+  for (int32_t t = blockIdx.x; t < n_units && ok; t += gridDim.x) {
+    const int32_t n[2] = {tile_info(p, t, 0).n_kv, tile_info(p, t, 1).n_kv};
+    const int32_t n_max = max(n[0], n[1]);
+    if (n_max == 0) continue;
+    if (!(ok = bwait(&ctl->q_full, u & 1, &ctl->abort, p))) break;
+    if (!(ok = wait_k(g))) break;
+    tc_fence_after();
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      if (n[s] > 0) {
+        pp_issue_s<Cfg>(tmem, qb[s], kbase(g), s);
+        tc_commit(&ctl->s_full[s]);
+      }
+    }
+    tc_commit(&ctl->k_empty[g % Cfg::kKStages]);
+    for (int32_t j = 1; j < n_max && ok; ++j) {
+      const uint32_t gk = g + j, gv = g + j - 1;
+      if (!(ok = wait_k(gk))) break;
+      if (!(ok = wait_v(gv))) break;
+#pragma unroll
+      for (int s = 0; s < 2; ++s) {
+        if (j - 1 < n[s] && !(ok = do_pv(s, j - 1, n[s], gv))) break;
+        if (j < n[s]) {
+          pp_issue_s<Cfg>(tmem, qb[s], kbase(gk), s);
+          tc_commit(&ctl->s_full[s]);
+        }
+      }
+      if (!ok) break;
+      tc_commit(&ctl->k_empty[gk % Cfg::kKStages]);
+      tc_commit(&ctl->v_empty[gv % Cfg::kVStages]);
+    }
+    if (!ok) break;
+    // All S products of this unit are issued: Q may be replaced once they finish.
+    tc_commit(&ctl->q_empty);
+    const uint32_t gl = g + n_max - 1;
+    if (!(ok = wait_v(gl))) break;
+#pragma unroll
+    for (int s = 0; s < 2; ++s)
+      if (n_max - 1 < n[s] && !(ok = do_pv(s, n_max - 1, n[s], gl))) break;
+    if (!ok) break;
+    tc_commit(&ctl->v_empty[gl % Cfg::kVStages]);
+    for (int s = 0; s < 2; ++s)
+      if (n[s] > 0) ++co[s];
+    g += n_max;
+    ++u;
+  }
+  tc_commit(&ctl->drain);
+  drain_wait(&ctl->drain, 0, p);
+}
+
+// ------------------------------------------------------------------- softmax
+template <int DV, int kEmuPer16>
+__device__ void pp_softmax(const AttnParams &p, PPCtrl *ctl, uint32_t tmem, int s) {
+  using T = __nv_bfloat16;
+  const int32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int32_t r = threadIdx.x & 127;                  // row within the tile = TMEM lane
+  const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+  const uint32_t s_addr = tmem + lane_base + (s ? 128u : 0u);
+  const uint32_t o_addr = tmem + lane_base + (s ? 384u : 256u);
+  const int32_t n_units = num_units(p);
+  uint32_t cs = 0, co = 0;
+  bool ok = true;
+  for (int32_t t = blockIdx.x; t < n_units && ok; t += gridDim.x) {
+    const TileInfo ti = tile_info(p, t, s);
+    const int32_t row = ti.q0 + r;
+    const bool row_valid = row < ti.lq;
+    if (ti.n_kv == 0) {
+      if (row_valid) store_zero_row<T, DV>(p, ti, row);
+      continue;
+    }
+    float m = -INFINITY, l = 0.f;
+    for (int32_t j = 0; j < ti.n_kv; ++j) {
+      if (!(ok = bwait(&ctl->s_full[s], cs & 1, &ctl->abort, p))) break;
+      ++cs;
+      tc_fence_after();
+      uint32_t sr[128];
+      tmem_ld_x128(s_addr, sr);
+      float x[128];
+      const float alpha = softmax_row<kEmuPer16>(p, ti, row, j * kBlockN, sr, x, m, l);
+      tmem_store_p<false>(s_addr, x);
+      // S_s(j) done implies PV_s(j-1) done: O_s may be rescaled right away.
+      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) tmem_scale_row<DV>(o_addr, alpha);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl->p_full[s]);
+    }
+    if (!ok) break;
+    if (!(ok = bwait(&ctl->o_full[s], co & 1, &ctl->abort, p))) break;
+    ++co;
+    tc_fence_after();
+    float o[DV];
+    tmem_load_row<DV>(o_addr, o);
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&ctl->o_empty[s]);
+    if (row_valid) store_row<T, DV>(p, ti, row, o, l > 0.f ? 1.f / l : 0.f);
+  }
+}
+
+// --------------------------------------------------------------------- kernel
+template <int DQK, int DROPE, int DV>
+__global__ void __launch_bounds__(kPPThreads, 1) attn_fwd_pp_kernel(const __grid_constant__ AttnParams p) {
+  using Cfg = PPCfg<DQK, DROPE, DV>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+  PPCtrl *ctl = reinterpret_cast<PPCtrl *>(smem + Cfg::kCtrlOff);
+  const int32_t warp = threadIdx.x >> 5;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&ctl->q_full, 1);
+    mbar_init(&ctl->q_empty, 1);
+    mbar_init(&ctl->drain, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&ctl->s_full[i], 1);
+      mbar_init(&ctl->p_full[i], 4);
+      mbar_init(&ctl->o_full[i], 1);
+      mbar_init(&ctl->o_empty[i], 4);
+    }
+    for (int i = 0; i < 3; ++i) {
+      mbar_init(&ctl->k_full[i], 1);
+      mbar_init(&ctl->k_empty[i], 1);
+      mbar_init(&ctl->v_full[i], 1);
+      mbar_init(&ctl->v_empty[i], 1);
+    }
+    ctl->abort = 0;
+    mbar_fence_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(&ctl->tmem_base, Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl->tmem_base;
+
+  ProducerLog plog;
+  if (warp < 8) {
+    regs_increase<kPPSoftmaxRegs>();
+    pp_softmax<DV, Cfg::kEmuPer16>(p, ctl, tmem, warp >> 2);
+  } else {
+    regs_decrease<kPPOtherRegs>();
+    if (warp == 8 && (threadIdx.x & 31) == 0) pp_producer<Cfg>(p, smem, ctl, plog);
+    if (warp == 9 && (threadIdx.x & 31) == 0) pp_mma<Cfg>(p, smem, ctl, tmem);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, Cfg::kTmemCols);
+  } else if (warp == 8 && (threadIdx.x & 31) == 0) {
+    if (plog.q_last >= 0) drain_wait(&ctl->q_full, plog.q_last & 1, p);
+    for (int s = 0; s < Cfg::kKStages; ++s)
+      if (plog.k_last[s] >= 0) drain_wait(&ctl->k_full[s], plog.k_last[s] & 1, p);
+    for (int s = 0; s < Cfg::kVStages; ++s)
+      if (plog.v_last[s] >= 0) drain_wait(&ctl->v_full[s], plog.v_last[s] & 1, p);
+  }
+}
+
+template <int DQK, int DROPE, int DV>
+cudaError_t launch_attn_pp(const AttnParams &p, int grid, cudaStream_t stream) {
+  using Cfg = PPCfg<DQK, DROPE, DV>;
+  auto kern = attn_fwd_pp_kernel<DQK, DROPE, DV>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       Cfg::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kPPThreads, Cfg::kSmemBytes, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace wf

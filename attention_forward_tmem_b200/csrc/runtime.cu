@@ -312,8 +312,8 @@ wf_status_t wf_attn_fwd_debug(const wf_tensor_t *q, const wf_tensor_t *qRope, co
   // supported head sizes
   if (d.drope && !(d.drope == 64 && d.dqk == 128 && d.dv == 128 && dt == WF_BF16))
     return fail(WF_ERR_UNSUPPORTED, "rope part needs bf16, Dqk = Dv = 128 and a 64-wide rope");
-  AttnLaunchFn launch = find_attn_kernel(dt == WF_BF16 ? 1 : 0, (int)d.dqk, (int)d.drope, (int)d.dv);
-  if (!launch)
+  const AttnKernel kern = find_attn_kernel(dt == WF_BF16 ? 1 : 0, (int)d.dqk, (int)d.drope, (int)d.dv);
+  if (!kern.launch)
     return fail(WF_ERR_UNSUPPORTED, "head sizes Dqk=%lld Dv=%lld (rope %lld) are not implemented",
                 (long long)d.dqk, (long long)d.dv, (long long)d.drope);
 
@@ -328,38 +328,33 @@ wf_status_t wf_attn_fwd_debug(const wf_tensor_t *q, const wf_tensor_t *qRope, co
 
   AttnParams p;
   std::memset(&p, 0, sizeof(p));
-  const int64_t es = (int64_t)dtype_size(dt);
-  (void)es;
-  // q / k / v maps: (D, rows, heads, batch)
-  if (!d.varlen) {
-    st = make_map(&p.tm_q, q->data, dt, d.dqk, d.lq, headNum, d.batch, q->stride[2], q->stride[1], q->stride[0], "q");
-    if (st == WF_OK)
-      st = make_map(&p.tm_k, k->data, dt, d.dqk, d.lk > 0 ? d.lk : 1, kvHeadNum, d.batch, k->stride[2], k->stride[1], k->stride[0], "k");
-    if (st == WF_OK)
-      st = make_map(&p.tm_v, v->data, dt, d.dv, d.lk > 0 ? d.lk : 1, kvHeadNum, d.batch, v->stride[2], v->stride[1], v->stride[0], "v");
-    if (st == WF_OK && d.drope) {
-      st = make_map(&p.tm_qr, qRope->data, dt, d.drope, d.lq, headNum, d.batch, qRope->stride[2], qRope->stride[1], qRope->stride[0], "qRope");
-      if (st == WF_OK)
-        st = make_map(&p.tm_kr, kRope->data, dt, d.drope, d.lk > 0 ? d.lk : 1, kvHeadNum, d.batch, kRope->stride[2], kRope->stride[1], kRope->stride[0], "kRope");
-    }
-  } else {
-    const int64_t tk = d.tk > 0 ? d.tk : 1;
-    st = make_map(&p.tm_q, q->data, dt, d.dqk, d.tq, headNum, 1, q->stride[0], q->stride[1], q->stride[0] * d.tq, "q");
-    if (st == WF_OK)
-      st = make_map(&p.tm_k, k->data, dt, d.dqk, tk, kvHeadNum, 1, k->stride[0], k->stride[1], k->stride[0] * tk, "k");
-    if (st == WF_OK)
-      st = make_map(&p.tm_v, v->data, dt, d.dv, tk, kvHeadNum, 1, v->stride[0], v->stride[1], v->stride[0] * tk, "v");
-    if (st == WF_OK && d.drope) {
-      st = make_map(&p.tm_qr, qRope->data, dt, d.drope, d.tq, headNum, 1, qRope->stride[0], qRope->stride[1], qRope->stride[0] * d.tq, "qRope");
-      if (st == WF_OK)
-        st = make_map(&p.tm_kr, kRope->data, dt, d.drope, tk, kvHeadNum, 1, kRope->stride[0], kRope->stride[1], kRope->stride[0] * tk, "kRope");
-    }
+  const int64_t n_keys = d.varlen ? d.tk : d.lk;   // rows of k / v
+  // q / k / v maps: (D, rows, heads, batch).  Dense: rows = sequence
+  // positions, batch = B.  Packed: rows = tokens of all sequences, batch = 1.
+  struct MapArgs { int64_t rows, batch, s_row, s_head, s_batch; };
+  auto dims_of = [&](const wf_tensor_t *t, int64_t rows) -> MapArgs {
+    if (!d.varlen) return {rows, d.batch, t->stride[2], t->stride[1], t->stride[0]};
+    return {rows, 1, t->stride[0], t->stride[1], t->stride[0] * rows};
+  };
+  auto map_of = [&](CUtensorMap *m, const wf_tensor_t *t, int64_t dd, int64_t rows, int64_t heads,
+                    const char *name) {
+    const MapArgs a = dims_of(t, rows);
+    return make_map(m, t->data, dt, dd, a.rows, heads, a.batch, a.s_row, a.s_head, a.s_batch, name);
+  };
+  const int64_t n_q = d.varlen ? d.tq : d.lq;
+  st = map_of(&p.tm_q, q, d.dqk, n_q, headNum, "q");
+  if (st == WF_OK && d.drope) st = map_of(&p.tm_qr, qRope, d.drope, n_q, headNum, "qRope");
+  if (st == WF_OK && n_keys > 0) {
+    st = map_of(&p.tm_k, k, d.dqk, n_keys, kvHeadNum, "k");
+    if (st == WF_OK && dt == WF_BF16) st = map_of(&p.tm_v, v, d.dv, n_keys, kvHeadNum, "v");
+    if (st == WF_OK && d.drope) st = map_of(&p.tm_kr, kRope, d.drope, n_keys, kvHeadNum, "kRope");
   }
   if (st != WF_OK) return st;
-  if (!d.drope) {   // unused maps: copies of q / k so the descriptor is well formed
-    p.tm_qr = p.tm_q;
-    p.tm_kr = p.tm_k;
-  }
+  // Maps that are never read (no rope part, or no key at all): copies of q's
+  // so that every descriptor passed to the kernel is well formed.
+  if (!d.drope) p.tm_qr = p.tm_q;
+  if (n_keys == 0) p.tm_k = p.tm_v = p.tm_q;
+  if (!d.drope || n_keys == 0) p.tm_kr = p.tm_k;
 
   p.out = out->data;
   if (!d.varlen) {
@@ -388,39 +383,69 @@ wf_status_t wf_attn_fwd_debug(const wf_tensor_t *q, const wf_tensor_t *qRope, co
   p.timeout_cycles = timeout_cycles > 0 ? timeout_cycles : (2LL << 30);
   p.debug_flags = debug_flags;
 
-  int grid = ds->sm_count;
-  if (!d.varlen) {
-    p.lq = (int32_t)d.lq;
-    p.lk = (int32_t)d.lk;
-    const int64_t nqt = (d.lq + kBlockM - 1) / kBlockM;
-    const int64_t tiles = nqt * d.batch * headNum;
-    if (tiles > INT32_MAX) return fail(WF_ERR_UNSUPPORTED, "too many tiles (%lld)", (long long)tiles);
-    p.nqt_dense = (int32_t)nqt;
-    p.n_tiles_dense = (int32_t)tiles;
-    if (tiles < grid) grid = (int)tiles;
-  } else {
-    // schedule workspace
+  // Per-stream workspace: [schedule tables (varlen)] [V^T (fp32)], 256-byte aligned parts.
+  SchedLayout sl{};
+  size_t sched_bytes = 0;
+  if (d.varlen) {
     const int64_t B = d.batch;
-    const int64_t cap = (d.tq + kBlockM - 1) / kBlockM + B;
+    const int64_t cap = (d.tq + kern.unit_rows - 1) / kern.unit_rows + B;
     if (cap * headNum > INT32_MAX) return fail(WF_ERR_UNSUPPORTED, "too many tiles");
-    SchedLayout sl;
     sl.cu_q = 2;
     sl.cu_k = (int32_t)(sl.cu_q + B + 1);
     sl.cu_t = (int32_t)(sl.cu_k + B + 1);
     sl.entries = (int32_t)(((sl.cu_t + B + 1) + 3) & ~int64_t(3));
     sl.capacity = (int32_t)cap;
     sl.words = sl.entries + 2 * cap;
-    int32_t *ws = nullptr;
-    if ((st = stream_workspace(dev, cs, (size_t)sl.words * 4, &ws)) != WF_OK) return st;
+    sched_bytes = ((size_t)sl.words * 4 + 255) & ~size_t(255);
+  }
+  const int64_t vt_ld = (n_keys + 3) & ~int64_t(3);
+  const int64_t vt_batch = d.varlen ? 1 : d.batch;
+  const size_t vt_bytes = dt == WF_F32 ? (size_t)(vt_batch * kvHeadNum * d.dv * vt_ld) * 4 : 0;
+  int32_t *ws = nullptr;
+  if (sched_bytes + vt_bytes > 0 &&
+      (st = stream_workspace(dev, cs, sched_bytes + vt_bytes, &ws)) != WF_OK)
+    return st;
+  if (dt == WF_F32) {
+    float *vt = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(ws) + sched_bytes);
+    if (n_keys > 0) {
+      const int64_t s_row = d.varlen ? v->stride[0] : v->stride[2];
+      const int64_t s_head = v->stride[1];
+      const int64_t s_batch = d.varlen ? 0 : v->stride[0];
+      cudaError_t e = launch_transpose_v(static_cast<const float *>(v->data), s_row, s_head, s_batch,
+                                         (int32_t)n_keys, kvHeadNum, (int32_t)vt_batch, (int32_t)d.dv,
+                                         vt, vt_ld, cs);
+      if (e != cudaSuccess) return cuda_fail(e, "V transpose launch");
+      // V^T as (keys, Dv rows, heads, batch): the kernel loads (128-byte key span) x 128 rows
+      st = make_map(&p.tm_v, vt, dt, n_keys, d.dv, kvHeadNum, vt_batch, vt_ld, d.dv * vt_ld,
+                    kvHeadNum * d.dv * vt_ld, "V^T");
+      if (st != WF_OK) return st;
+    } else {
+      p.tm_v = p.tm_q;    // never read: no key
+    }
+  }
+
+  int grid = ds->sm_count;
+  p.unit_rows = kern.unit_rows;
+  if (!d.varlen) {
+    p.lq = (int32_t)d.lq;
+    p.lk = (int32_t)d.lk;
+    const int64_t per_bh = (d.lq + kern.unit_rows - 1) / kern.unit_rows;
+    const int64_t units = per_bh * d.batch * headNum;
+    if (units > INT32_MAX) return fail(WF_ERR_UNSUPPORTED, "too many work units (%lld)", (long long)units);
+    p.units_per_bh = (int32_t)per_bh;
+    p.n_units_dense = (int32_t)units;
+    if (units < grid) grid = (int)units;
+  } else {
+    const int64_t B = d.batch;
     cudaError_t e = launch_sched_prep(static_cast<const int32_t *>(qSeqLen->data),
                                       static_cast<const int32_t *>(kvSeqLen->data), (int32_t)B,
-                                      d.tq, d.tk, maskType == WF_MASK_CAUSAL ? 1 : 0, ws, sl,
-                                      ds->status, cs);
+                                      d.tq, d.tk, maskType == WF_MASK_CAUSAL ? 1 : 0,
+                                      kern.unit_rows, ws, sl, ds->status, cs);
     if (e != cudaSuccess) return cuda_fail(e, "sched_prep launch");
     p.ws = ws;
     p.sl = sl;
   }
-  cudaError_t e = launch(p, grid, cs);
+  cudaError_t e = kern.launch(p, grid, cs);
   if (e != cudaSuccess) return cuda_fail(e, "attention kernel launch");
   return WF_OK;
 }

@@ -5,10 +5,11 @@
 // CTA of 1024 threads:
 //   1. prefix sums of the q lengths, kv lengths and q-tile counts;
 //   2. a length check (non-negative, sums within the tensors);
-//   3. the (sequence, q tile) entries ordered by KV-tile count, longest first
-//      (counting sort over the count), so the persistent attention CTAs take
-//      the long causal tiles first and finish together.
-// The attention kernel then maps work tile t to entry t / headNum and head
+//   3. the (sequence, work unit) entries ordered by the KV-tile count of the
+//      unit's last row, longest first (counting sort over the count), so the
+//      persistent attention CTAs take the long causal units first and finish
+//      together.  A work unit is `unit_rows` consecutive query rows.
+// The attention kernel then maps work item t to entry t / headNum and head
 // t % headNum, so the heads of one GQA group run next to each other.
 #include <cstdint>
 
@@ -49,16 +50,17 @@ __device__ int64_t block_exclusive_scan(int64_t v, int64_t &excl, int64_t *warp_
   return total;
 }
 
-__device__ __forceinline__ int32_t kv_tiles(int32_t q0, int32_t lq, int32_t lk, int32_t causal) {
+__device__ __forceinline__ int32_t kv_tiles(int32_t q0, int32_t rows, int32_t lq, int32_t lk,
+                                            int32_t causal) {
   int32_t kend = lk;
-  if (causal) kend = min(kend, min(q0 + kBlockM, lq) + (lk - lq));
+  if (causal) kend = min(kend, min(q0 + rows, lq) + (lk - lq));
   return kend > 0 ? (kend + kBlockN - 1) / kBlockN : 0;
 }
 
 __global__ void __launch_bounds__(kSchedThreads) sched_prep_kernel(
     const int32_t *__restrict__ q_len, const int32_t *__restrict__ k_len, int32_t batch,
     int64_t n_q_tokens, int64_t n_k_tokens, int32_t causal, int32_t *__restrict__ ws,
-    SchedLayout sl, int32_t *__restrict__ status) {
+    int32_t unit_rows, SchedLayout sl, int32_t *__restrict__ status) {
   __shared__ int64_t warp_tot[33];
   __shared__ int32_t hist[kHistBins];
   __shared__ int32_t bad;
@@ -78,7 +80,7 @@ __global__ void __launch_bounds__(kSchedThreads) sched_prep_kernel(
       lq = q_len[b];
       lk = k_len[b];
       if (lq < 0 || lk < 0) atomicOr(&bad, 1);
-      nt = lq > 0 ? (lq + kBlockM - 1) / kBlockM : 0;
+      nt = lq > 0 ? (lq + unit_rows - 1) / unit_rows : 0;
     }
     int64_t eq, ek, et;
     const int64_t tq = block_exclusive_scan(lq, eq, warp_tot);
@@ -128,7 +130,7 @@ __global__ void __launch_bounds__(kSchedThreads) sched_prep_kernel(
   auto bin_of = [&](int32_t b, int32_t qt) {
     const int32_t lq = ws[sl.cu_q + b + 1] - ws[sl.cu_q + b];
     const int32_t lk = ws[sl.cu_k + b + 1] - ws[sl.cu_k + b];
-    const int32_t w = kv_tiles(qt * kBlockM, lq, lk, causal);
+    const int32_t w = kv_tiles(qt * unit_rows, unit_rows, lq, lk, causal);
     return kHistBins - 1 - min(w, kHistBins - 1);
   };
   for (int32_t e = tid; e < n_entries; e += kSchedThreads) {
@@ -175,11 +177,11 @@ __global__ void __launch_bounds__(kSchedThreads) sched_prep_kernel(
 
 cudaError_t launch_sched_prep(const int32_t *q_len, const int32_t *k_len, int32_t batch,
                               int64_t n_q_tokens, int64_t n_k_tokens, int32_t causal,
-                              int32_t *ws, const SchedLayout &sl, int32_t *status,
-                              cudaStream_t stream) {
+                              int32_t unit_rows, int32_t *ws, const SchedLayout &sl,
+                              int32_t *status, cudaStream_t stream) {
   static_assert(kHistBins == 4 * kSchedThreads, "scan covers 4 bins per thread");
   sched_prep_kernel<<<1, kSchedThreads, 0, stream>>>(q_len, k_len, batch, n_q_tokens, n_k_tokens,
-                                                     causal, ws, sl, status);
+                                                     causal, ws, unit_rows, sl, status);
   return cudaGetLastError();
 }
 

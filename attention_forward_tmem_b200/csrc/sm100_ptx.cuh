@@ -203,12 +203,88 @@ __device__ __forceinline__ void tmem_st_x64(uint32_t taddr, const uint32_t (&r)[
       : "memory");
 }
 
+// --------------------------------------------------------- register split
+// Per-warpgroup register limits (all four warps of a warpgroup execute the
+// same one).  The sum over the CTA must stay within the registers the CTA was
+// launched with.
+template <uint32_t N>
+__device__ __forceinline__ void regs_increase() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_decrease() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ------------------------------------------------------------- math
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// max(a, b, c) in one instruction (sm_100 three-input form).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+// (d0, d1) = (a0 * b + c, a1 * b + c), one packed f32x2 FMA.
+__device__ __forceinline__ void fma2_bc(float &d0, float &d1, float a0, float a1, float b, float c) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %4};\n\tmov.b64 rc, {%5, %5};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b), "f"(c));
+}
+// (s0, s1) += (a0, a1), one packed f32x2 add.
+__device__ __forceinline__ void add2(float &s0, float &s1, float a0, float a1) {
+  asm("{\n\t.reg .b64 rs, ra;\n\t"
+      "mov.b64 rs, {%0, %1};\n\tmov.b64 ra, {%2, %3};\n\t"
+      "add.rn.f32x2 rs, rs, ra;\n\tmov.b64 {%0, %1}, rs;\n\t}"
+      : "+f"(s0), "+f"(s1)
+      : "f"(a0), "f"(a1));
+}
+// (d0, d1) = (a0 + b0, a1 + b1), one packed f32x2 add.
+__device__ __forceinline__ void add2_to(float &d0, float &d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+// (d0, d1) = (a0 * b0 + c0, a1 * b1 + c1), one packed f32x2 FMA.
+__device__ __forceinline__ void fma2_to(float &d0, float &d1, float a0, float a1, float b0, float b1,
+                                        float c0, float c1) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+
+// 2^x for two finite x on the FMA pipe (no MUFU): Cody-Waite reduction
+// x = n + f, n = round(x) (by adding 1.5 * 2^23, which leaves n in the low
+// mantissa bits), f in [-1/2, 1/2]; 2^f by a degree-3 minimax polynomial
+// (coefficients from exp2_poly_fit.py, max relative error 7.5e-5); n is added
+// to the exponent field of P(f).  Inputs are clamped to >= -125 so the
+// exponent never underflows (2^-125 instead of a smaller value), so this is
+// only used where no score is masked.
+__device__ __forceinline__ void exp2_poly2(float &a, float &b) {
+  constexpr float kShift = 12582912.0f;          // 1.5 * 2^23
+  constexpr float c0 = 0.99992806f, c1 = 0.69326097f, c2 = 0.24261113f, c3 = 0.05517167f;
+  const float xa = fmaxf(a, -125.f), xb = fmaxf(b, -125.f);
+  float ta, tb, ra, rb, fa, fb, pa, pb;
+  add2_to(ta, tb, xa, xb, kShift, kShift);        // round to nearest integer
+  add2_to(ra, rb, ta, tb, -kShift, -kShift);      // n as a float
+  add2_to(fa, fb, xa, xb, -ra, -rb);              // f = x - n
+  fma2_to(pa, pb, fa, fb, c3, c3, c2, c2);
+  fma2_to(pa, pb, pa, pb, fa, fb, c1, c1);
+  fma2_to(pa, pb, pa, pb, fa, fb, c0, c0);
+  // bits(t) = 0x4B400000 + n, and 0x4B400000 << 23 vanishes mod 2^32
+  a = __int_as_float(__float_as_int(pa) + (__float_as_int(ta) << 23));
+  b = __int_as_float(__float_as_int(pb) + (__float_as_int(tb) << 23));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&v);

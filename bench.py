@@ -1,0 +1,404 @@
+"""Benchmark of the attention forward on B200 (one JSON line on stdout).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+A step is one call of the library's attention forward over one batch of the
+workload (for ``gqa_causal_prefill``: B 4, 32 query / 8 kv heads, L 4096, D 128,
+bf16, causal).  Inputs are synthetic (seeded N(0,1)), resident in HBM before
+the timed region; their footprint (335 MB) is larger than L2, so no flush is
+needed between steps.  Timing: W untimed steps, barrier + synchronize, CUDA
+events around exactly K steps on the launching stream, synchronize, max over
+ranks.  The metric is FLOP/s with causal-adjusted (kept-pair) FLOPs:
+sum over (b, h) of 2 * (Dqk + Dv) * kept pairs.
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own copy of the
+workload (independent batches: weak scaling, no collective on the data path);
+`value` = all ranks' FLOPs / the slowest rank's time.
+
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same
+workload (rank 0 only), the slow baseline arm.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from attention_forward_tmem_b200 import workloads as W  # noqa: E402
+
+METRIC = "attention fwd TFLOP/s (causal-adjusted) and % of B200 dense BF16 tensor peak"
+DATASHEET_BF16_TFLOPS = 2250.0        # NVIDIA B200 dense BF16, for the second peak reading
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ["attention_forward_tmem_b200/csrc/attn_kernel.cuh",
+                  "attention_forward_tmem_b200/csrc/sm100_ptx.cuh",
+                  "attention_forward_tmem_b200/csrc/attn_params.h"]
+
+
+# ----------------------------------------------------------------- helpers
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def kernel_hash():
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload):
+    """DRAM bytes per launch from the committed ncu summary of this workload,
+    if it was taken on the current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", f"attn_fwd_{workload}.md")
+    if not os.path.exists(p):
+        return None
+    txt = open(p).read()
+    mh = re.search(r"kernel_source_hash:\s*([0-9a-f]+)", txt)
+    mt = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", txt)
+    if not mh or not mt or mh.group(1) != kernel_hash():
+        return None
+    return float(mt.group(1))
+
+
+def kept_pairs_causal(lq, lk):
+    """Kept (query, key) pairs of one head under the bottom-right causal mask."""
+    off = lk - lq
+    total = 0
+    for i in range(lq):
+        total += max(0, min(lk, i + off + 1))
+    return total
+
+
+class ClockSampler:
+    """Polls NVML (SM clock, clock-event reasons) every 10 ms on a thread."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, device_index):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            try:
+                self.h = pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + uuid).encode())
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # pragma: no cover - NVML missing
+            self.err = str(e)
+        self._stop = threading.Event()
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            self._stop.wait(0.01)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "NVML unavailable"}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------- workloads
+
+class Workload:
+    """One step's inputs and the call that runs it through the public API."""
+
+    def __init__(self, name, device):
+        from attention_forward_tmem_b200 import api
+        self.api = api
+        self.name = name
+        self.device = device
+        w = W.WORKLOADS[name]
+        self.w = w
+        self.launches_per_step = 1
+        if name in ("gqa_causal_prefill", "long_gqa_causal"):
+            q, k, v = W.dense_inputs(w.batch, w.head_num, w.kv_head_num, w.seq, w.seq, w.dqk, w.dv,
+                                     w.dtype, W.SEED, w.input_scale)
+            self.host = {"q": q, "k": k, "v": v}
+            self.flops = w.batch * w.head_num * 2 * (w.dqk + w.dv) * kept_pairs_causal(w.seq, w.seq)
+            self.config = {"workload": name, "batch": w.batch, "head_num": w.head_num,
+                           "kv_head_num": w.kv_head_num, "seq_len": w.seq, "head_dim": w.dqk,
+                           "mask": "causal"}
+        elif name == "mla_varlen_prefill":
+            d = W.mla_varlen_prefill()
+            self.host = d
+            lens = d["q_seqlen"].tolist()
+            self.flops = sum(w.head_num * 2 * (w.dqk + w.drope + w.dv) * kept_pairs_causal(L, L)
+                             for L in lens)
+            self.launches_per_step = 2          # schedule + attention
+            self.config = {"workload": name, "batch": w.batch, "seqlens": lens,
+                           "n_tokens": int(sum(lens)), "head_num": w.head_num,
+                           "head_dim": w.dqk, "rope_dim": w.drope, "mask": "causal"}
+        else:
+            raise SystemExit(f"bench workload {name!r} is not a single-call workload")
+        self.out_host = None
+
+    def to_device(self):
+        self.dev = {k: v.to(self.device) for k, v in self.host.items()}
+        self.out = self._alloc_out()
+
+    def _alloc_out(self):
+        q = self.dev["q"]
+        if self.name == "mla_varlen_prefill":
+            return torch.empty(q.shape[0], q.shape[1], self.w.dv, dtype=q.dtype, device=self.device)
+        return torch.empty(q.shape[:3] + (self.w.dv,), dtype=q.dtype, device=self.device)
+
+    def step(self, dev=None, out=None):
+        d = dev or self.dev
+        kw = dict(mask_type=self.api.MaskType.CAUSAL, qk_scale=self.w.qk_scale, out=out or self.out)
+        if self.name == "mla_varlen_prefill":
+            kw.update(qrope=d["qrope"], krope=d["krope"], q_seqlen=d["q_seqlen"],
+                      kv_seqlen=d["kv_seqlen"])
+        self.api.attn_fwd(d["q"], d["k"], d["v"], **kw)
+
+    def host_bytes(self):
+        return sum(t.numel() * t.element_size() for t in self.host.values())
+
+
+def time_device(wl, steps, warmup, dist_on):
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        wl.step()
+    torch.cuda.synchronize()
+    if dist_on:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        e0.record(stream)
+        for _ in range(steps):
+            wl.step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    wl.api.device_status()
+    return ms, clk.summary()
+
+
+def time_e2e(wl, steps, warmup):
+    """Same steps through the public API with host inputs: pinned host -> device
+    copies of q/k/v (+lengths) and the device -> host copy of the output are
+    inside the timed region."""
+    pinned = {k: v.pin_memory() for k, v in wl.host.items()}
+    out_host = torch.empty(wl.out.shape, dtype=wl.out.dtype).pin_memory()
+    dev = {k: torch.empty_like(v, device=wl.device) for k, v in pinned.items()}
+    stream = torch.cuda.current_stream()
+
+    def one():
+        for k in pinned:
+            dev[k].copy_(pinned[k], non_blocking=True)
+        wl.step(dev=dev)
+        out_host.copy_(wl.out, non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    h2d = sum(t.numel() * t.element_size() for t in pinned.values())
+    d2h = out_host.numel() * out_host.element_size()
+    return e0.elapsed_time(e1), h2d, d2h
+
+
+# -------------------------------------------------------------- CPU oracle
+
+def oracle_sample(name, budget_s=12.0, seed=7):
+    """Time the fp64 oracle on rows of the workload (each over its full key
+    range) for about `budget_s` seconds.  Returns (TFLOP/s, threads, note)."""
+    import oracle
+    w = W.WORKLOADS[name]
+    rng = np.random.default_rng(seed)
+    if name == "mla_varlen_prefill":
+        raise SystemExit("cpu baseline is defined for the dense workloads")
+    # one GQA group of one batch entry: q [1, G, L, D], k/v [1, 1, L, D]
+    g = w.head_num // w.kv_head_num
+    q, k, v = W.dense_inputs(1, g, 1, w.seq, w.seq, w.dqk, w.dv, w.dtype, seed, w.input_scale)
+
+    def run(n_rows):
+        rows = np.stack([np.zeros(n_rows, np.int64), rng.integers(0, g, n_rows),
+                         rng.integers(0, w.seq, n_rows)], 1)
+        fl = float(sum(2 * (w.dqk + w.dv) * (int(r) + 1) for r in rows[:, 2]))
+        t0 = time.perf_counter()
+        oracle.sdpa_rows(q, k, v, rows, mask_kind="causal", qk_scale=w.qk_scale,
+                         head_num=g, kv_head_num=1)
+        return fl, time.perf_counter() - t0
+
+    fl, dt = run(64)                           # calibrate
+    rate = fl / max(dt, 1e-6)
+    n = int(min(200000, max(64, rate * budget_s / (2 * (w.dqk + w.dv) * w.seq / 2))))
+    fl, dt = run(n)
+    note = (f"{n} query rows of {name} (one GQA group, rows uniform in [0, {w.seq}), "
+            f"each over its full causal key range), fp64 oracle, {dt:.1f} s")
+    return fl / dt / 1e12, oracle.oracle_threads(), note
+
+
+# -------------------------------------------------------------------- main
+
+def dist_setup(args):
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    if ws > 1:
+        import datetime
+        local = int(os.environ.get("LOCAL_RANK", "0"))
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+        return True, torch.distributed.get_rank(), ws
+    if args.gpus > 1:
+        raise SystemExit("--gpus > 1 needs torchrun (one process per GPU)")
+    return False, 0, 1
+
+
+def reference_arm(args, rank, world):
+    if rank != 0:
+        return
+    name = args.workload
+    w = W.WORKLOADS[name]
+    per_step = []
+    note = threads = None
+    for i in range(args.warmup + args.steps):
+        v, threads, note = oracle_sample(name, budget_s=args.ref_step_s, seed=100 + i)
+        if i >= args.warmup:
+            per_step.append(v)
+    val = statistics.mean(per_step)
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": name, "batch": w.batch, "head_num": w.head_num,
+                       "kv_head_num": w.kv_head_num, "seq_len": w.seq, "head_dim": w.dqk,
+                       "mask": w.mask, "parallelism": "host cores"},
+            "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                             "sample": note},
+            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="gqa_causal_prefill",
+                    choices=["gqa_causal_prefill", "mla_varlen_prefill", "long_gqa_causal"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-step-s", type=float, default=3.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be at least 3")
+
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        reference_arm(args, rank, int(os.environ.get("WORLD_SIZE", "1")))
+        return
+
+    dist_on, rank, world = dist_setup(args)
+    device = torch.device("cuda", torch.cuda.current_device())
+    wl = Workload(args.workload, device)
+    wl.to_device()
+
+    ms, clocks = time_device(wl, args.steps, args.warmup, dist_on)
+    if dist_on:
+        t = torch.tensor([ms], device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    per_launch_ms = ms / args.steps
+    value = wl.flops * world * args.steps / (ms / 1e3) / 1e12
+
+    e2e_ms, h2d, d2h = time_e2e(wl, max(3, min(args.steps, 20)), 3)
+    e2e_steps = max(3, min(args.steps, 20))
+    if dist_on:
+        t = torch.tensor([e2e_ms], device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_val = wl.flops * world * e2e_steps / (e2e_ms / 1e3) / 1e12
+
+    peaks, peak_kind = measured_peaks()
+    achieved = wl.flops / (per_launch_ms / 1e3) / 1e12
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                "traffic": profiled_traffic(args.workload),
+                "peak_source": f"{peak_kind} bf16 burst (MEASURED_PEAKS.json)"
+                if peak_kind == "measured" else "fallback 1.59 PFLOP/s",
+                "kernel": "wf::attn_fwd_kernel", "algorithmic_flops_per_launch": wl.flops}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload != "mla_varlen_prefill":
+        v, threads, note = oracle_sample(args.workload)
+        cpu = {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": note}
+
+    if dist_on:
+        torch.distributed.barrier()
+    if rank == 0:
+        cfg = dict(wl.config)
+        cfg["parallelism"] = f"dp{world}" if world > 1 else "single GPU"
+        cfg["l2"] = f"inputs larger than L2 ({wl.host_bytes() / 1e6:.0f} MB + output)"
+        line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_launch_ms,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic (seeded N(0,1), see workloads.py)",
+                "config": cfg,
+                "pct_of_peak": {"measured_bf16": 100 * achieved / peaks["bf16_tflops"],
+                                "datasheet_bf16_2250": 100 * achieved / DATASHEET_BF16_TFLOPS},
+                "roofline": roofline, "cpu_baseline": cpu,
+                "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                        "d2h_bytes_per_step": d2h},
+                "clocks": clocks,
+                "gpu_launches": args.steps * wl.launches_per_step}
+        print(json.dumps(line), flush=True)
+    if dist_on:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
