@@ -44,6 +44,8 @@ SIGNATURES = {
     "wf_attn_fwd": (_I32, [_T, _T, _T, _T, _T, _T, _T, _T, _I32, _I32, _F32, _I32, _T, _P]),
     "wf_attn_fwd_debug": (_I32, [_T, _T, _T, _T, _T, _T, _T, _T, _I32, _I32, _F32, _I32, _T, _P,
                                  _U32, _I64]),
+    "wf_attn_fwd_varlen_noalloc": (_I32, [_T, _T, _T, _T, _T, _T, _T, _I32, _I32, _F32, _I32, _T,
+                                          _P]),
     "wf_kvcache_create": (_I32, [_T, _T, _I32, _I64, _I64, _I64, ctypes.POINTER(_P)]),
     "wf_kvcache_before_update": (_I32, [_P, _I64]),
     "wf_kvcache_update": (_I32, [_P, _T, _T, _P]),

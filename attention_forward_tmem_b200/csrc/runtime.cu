@@ -128,7 +128,7 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // 4-d map (D, rows, heads, batch) with a (128 B of D) x 128 rows box, 128-byte
 // swizzle, zero fill outside the tensor.  Strides in elements.
-static wf_status_t make_map(CUtensorMap *map, const void *base, int32_t dtype, int64_t d,
+wf_status_t make_map(CUtensorMap *map, const void *base, int32_t dtype, int64_t d,
                             int64_t rows, int64_t heads, int64_t batch, int64_t s_row,
                             int64_t s_head, int64_t s_batch, const char *name) {
   auto fn = encode_fn();
@@ -152,7 +152,7 @@ static wf_status_t make_map(CUtensorMap *map, const void *base, int32_t dtype, i
 // ------------------------------------------------------------- validation
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-static int64_t numel(const wf_tensor_t *t) {
+int64_t numel(const wf_tensor_t *t) {
   int64_t n = 1;
   for (int i = 0; i < t->ndim; ++i) n *= t->shape[i];
   return n;
@@ -160,8 +160,8 @@ static int64_t numel(const wf_tensor_t *t) {
 
 // Basic descriptor checks: ndim, dtype, non-negative shape, last stride 1,
 // 16-byte alignment of the base and of every other stride.
-static wf_status_t check_tensor(const wf_tensor_t *t, const char *name, int ndim, int32_t dtype,
-                                bool need_tma_layout) {
+wf_status_t check_tensor(const wf_tensor_t *t, const char *name, int ndim, int32_t dtype,
+                         bool need_tma_layout) {
   if (!t) return fail(WF_ERR_INVALID_ARG, "%s is NULL", name);
   if (t->ndim != ndim) return fail(WF_ERR_INVALID_ARG, "%s: expected %d dims, got %d", name, ndim, t->ndim);
   if (t->dtype != dtype)

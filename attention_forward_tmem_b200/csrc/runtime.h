@@ -4,6 +4,8 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include <cuda.h>
+
 #include "wf_attn.h"
 
 namespace wf {
@@ -27,7 +29,14 @@ struct DeviceState {
 };
 // Current device's state (lazily initialised), or nullptr with the error set.
 DeviceState *current_device_state(wf_status_t *st);
-// Grow the current device's workspace to at least `bytes`.
-wf_status_t ensure_workspace(DeviceState *ds, size_t bytes);
+// Tensor helpers shared by the entry points (runtime.cu).
+wf_status_t check_tensor(const wf_tensor_t *t, const char *name, int ndim, int32_t dtype,
+                         bool need_tma_layout);
+int64_t numel(const wf_tensor_t *t);
+// 4-d TMA map (D, rows, heads, batch), (128 bytes of D) x 128 rows box,
+// 128-byte swizzle, zero fill outside the tensor; strides in elements.
+wf_status_t make_map(CUtensorMap *map, const void *base, int32_t dtype, int64_t d, int64_t rows,
+                     int64_t heads, int64_t batch, int64_t s_row, int64_t s_head, int64_t s_batch,
+                     const char *name);
 
 }  // namespace wf

@@ -156,6 +156,33 @@ wf_status_t wf_attn_fwd_debug(const wf_tensor_t *q, const wf_tensor_t *qRope,
                               int32_t maskType, wf_tensor_t *out, void *stream,
                               uint32_t debug_flags, int64_t timeout_cycles);
 
+/*
+ * wf_attn_fwd_varlen_noalloc -- the packed-sequence (varlen) bf16 form of
+ * wf_attn_fwd that never allocates memory.  The pages have no counterpart;
+ * it exists for callers that cannot call cudaMalloc once they run (work
+ * captured into CUDA graphs that must leave the allocator alone, runtimes
+ * that give the whole device to a pool at start-up, fixed memory budgets).
+ *
+ * Arguments as in wf_attn_fwd's packed layout (no mask; maskType NONE or
+ * CAUSAL; all tensors WF_BF16).  Instead of an allocated workspace, the
+ * schedule tables live in a fixed array inside the library: 65536 int32
+ * words (256 KiB) on every GPU that loads the library, held until the
+ * process exits.  A call needs 3 * (batch + 1) + 2 * (ceil(nTokens / 256) +
+ * batch) + 8 words; larger calls return WF_ERR_INVALID_ARG and launch
+ * nothing.  The first call on a device looks the array's address up
+ * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * All calls share the array: calls whose work overlaps on the GPU (e.g. on
+ * different streams) race; calls in order on one stream do not, as each
+ * rewrites every word it reads.  Other dtypes and the dense layout return
+ * WF_ERR_UNSUPPORTED (the dense bf16 path of wf_attn_fwd allocates nothing).
+ */
+wf_status_t wf_attn_fwd_varlen_noalloc(const wf_tensor_t *q, const wf_tensor_t *qRope,
+                                       const wf_tensor_t *k, const wf_tensor_t *kRope,
+                                       const wf_tensor_t *v,
+                                       const wf_tensor_t *qSeqLen, const wf_tensor_t *kvSeqLen,
+                                       int32_t headNum, int32_t kvHeadNum, float qkScale,
+                                       int32_t maskType, wf_tensor_t *out, void *stream);
+
 /* ---------------------------------------------------------------------------
  * BlockKVCache ([P1] "Block KV cache 的调用顺序").
  *
