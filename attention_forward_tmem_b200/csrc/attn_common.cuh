@@ -29,41 +29,51 @@ struct TileInfo {
   int32_t b, h, hk, q0, lq, lk, qrow, krow, n_kv, off, tma_b;
 };
 
-// Sub-tile `sub` (128 rows each) of work unit `t`.  Dense units are ordered
-// longest causal range first; packed units come from the schedule table.
+// Sub-tile `sub` (128 rows each) of work item `t`; the enumeration order is
+// described in attn_params.h (per sequence, per kv head, longest unit first,
+// GQA heads adjacent).
 __device__ __forceinline__ TileInfo tile_info(const AttnParams &p, int32_t t, int32_t sub) {
   TileInfo ti;
-  int32_t u;
+  const int32_t G = p.group;
+  const bool causal = p.mask_kind == kMaskCausal;
+  int32_t r, n_units;
   if (!p.varlen) {
-    const int32_t bh = p.batch * p.hq;
-    u = p.units_per_bh - 1 - t / bh;
-    const int32_t r = t % bh;
-    ti.b = r / p.hq;
-    ti.h = r % p.hq;
+    n_units = p.units_per_bh;
+    const int32_t per_bhk = n_units * G;                // items of one (batch, kv head)
+    const int32_t blk = t / per_bhk;
+    r = t - blk * per_bhk;
+    ti.b = blk / p.hkv;
+    ti.hk = blk - ti.b * p.hkv;
     ti.lq = p.lq;
     ti.lk = p.lk;
     ti.krow = 0;
     ti.tma_b = ti.b;
-    ti.q0 = u * p.unit_rows + sub * kBlockM;
-    ti.qrow = ti.q0;
   } else {
-    const int32_t e = t / p.hq;
-    ti.h = t % p.hq;
-    const int32_t *ent = p.ws + p.sl.entries + 2 * e;
-    ti.b = __ldg(ent);
-    u = __ldg(ent + 1);
+    const int32_t *cu_work = p.ws + p.sl.cu_work;
+    int32_t lo = 0, hi = p.batch - 1;                   // last k with cu_work[k] <= t
+    while (lo < hi) {
+      const int32_t mid = (lo + hi + 1) >> 1;
+      if (__ldg(cu_work + mid) <= t) lo = mid; else hi = mid - 1;
+    }
+    ti.b = __ldg(p.ws + p.sl.order + lo);
+    r = t - __ldg(cu_work + lo);
     const int32_t cq = __ldg(p.ws + p.sl.cu_q + ti.b), ck = __ldg(p.ws + p.sl.cu_k + ti.b);
     ti.lq = __ldg(p.ws + p.sl.cu_q + ti.b + 1) - cq;
     ti.lk = __ldg(p.ws + p.sl.cu_k + ti.b + 1) - ck;
     ti.krow = ck;
     ti.tma_b = 0;
-    ti.q0 = u * p.unit_rows + sub * kBlockM;
-    ti.qrow = cq + ti.q0;
+    n_units = (ti.lq + p.unit_rows - 1) / p.unit_rows;
+    ti.hk = r / (n_units * G);
+    r -= ti.hk * n_units * G;
   }
-  ti.hk = ti.h / p.group;
+  const int32_t j = r / G;
+  ti.h = ti.hk * G + (r - j * G);
+  const int32_t u = causal ? n_units - 1 - j : j;
+  ti.q0 = u * p.unit_rows + sub * kBlockM;
+  ti.qrow = (p.varlen ? __ldg(p.ws + p.sl.cu_q + ti.b) : 0) + ti.q0;
   ti.off = ti.lk - ti.lq;
   int32_t kend = ti.q0 < ti.lq ? ti.lk : 0;            // no valid row: nothing to do
-  if (p.mask_kind == kMaskCausal) {
+  if (causal) {
     const int32_t last = min(ti.q0 + kBlockM, ti.lq);   // one past the last valid row
     kend = min(kend, last + ti.off);
   }
@@ -73,7 +83,7 @@ __device__ __forceinline__ TileInfo tile_info(const AttnParams &p, int32_t t, in
 
 __device__ __forceinline__ int32_t num_units(const AttnParams &p) {
   if (!p.varlen) return p.n_units_dense;
-  return __ldg(p.ws) * p.hq;
+  return __ldg(p.ws);
 }
 
 // Bounded wait.  Returns false (and raises the CTA abort flag) on expiry, or

@@ -21,14 +21,20 @@ constexpr int32_t kDevTimeout = 6;
 // Debug switches for the bounded-wait test entry point (0 in production).
 constexpr uint32_t kDebugStarveFirstK = 1u;   // producer never loads the first K tile
 
-// Varlen schedule workspace (int32 words):
-//   [0] number of (sequence, q-tile) entries E, [1] length-check flag,
+// Work order.  A work item is (sequence b, query head h, unit u), a unit being
+// `unit_rows` consecutive query rows.  Items are enumerated sequence by
+// sequence (packed: longest sequence first), then by kv head, then by unit
+// (causal: the longest unit first), with the query heads of one GQA group
+// adjacent: the items running at the same time on the 148 SMs then share
+// few K/V tensors, which stay in L2, and the short units come last.
+//
+// Packed-sequence schedule workspace (int32 words), written by sched_prep:
+//   [0] number of work items, [1] length-check flag,
 //   [cu_q .. cu_q+B] and [cu_k .. cu_k+B] prefix sums of the lengths,
-//   [cu_t .. cu_t+B] prefix sums of work units per sequence,
-//   [entries ..] E pairs (sequence, unit), longest KV range first.
-// A work unit is `unit_rows` consecutive query rows of one sequence.
+//   [order .. order+B) sequences by unit count, longest first,
+//   [cu_work .. cu_work+B] prefix sums of (units x headNum) in that order.
 struct SchedLayout {
-  int32_t cu_q, cu_k, cu_t, entries, capacity;   // offsets in words; capacity in entries
+  int32_t cu_q, cu_k, order, cu_work;   // offsets in words
   int64_t words;
 };
 
@@ -69,7 +75,7 @@ cudaError_t launch_transpose_v(const float *v, int64_t s_row, int64_t s_head, in
                                int64_t ld, cudaStream_t stream);
 
 cudaError_t launch_sched_prep(const int32_t *q_len, const int32_t *k_len, int32_t batch,
-                              int64_t n_q_tokens, int64_t n_k_tokens, int32_t causal,
+                              int64_t n_q_tokens, int64_t n_k_tokens, int32_t head_num,
                               int32_t unit_rows, int32_t *ws, const SchedLayout &sl,
                               int32_t *status, cudaStream_t stream);
 

@@ -107,21 +107,20 @@ extern "C" wf_status_t wf_attn_fwd_varlen_noalloc(
   if (B == 0 || tq == 0) return WF_OK;
 
   // schedule layout (same as wf_attn_fwd) and the size limit of the array
-  const int64_t cap = (tq + kern.unit_rows - 1) / kern.unit_rows + B;
+  const int64_t max_items = ((tq + kern.unit_rows - 1) / kern.unit_rows + B) * headNum;
+  if (max_items > INT32_MAX) return fail(WF_ERR_UNSUPPORTED, "too many work items");
   SchedLayout sl{};
   sl.cu_q = 2;
   sl.cu_k = (int32_t)(sl.cu_q + B + 1);
-  sl.cu_t = (int32_t)(sl.cu_k + B + 1);
-  sl.entries = (int32_t)(((sl.cu_t + B + 1) + 3) & ~int64_t(3));
-  sl.capacity = (int32_t)cap;
-  sl.words = sl.entries + 2 * cap;
-  if (sl.words > kScheduleWords || cap * headNum > INT32_MAX)
+  sl.order = (int32_t)(sl.cu_k + B + 1);
+  sl.cu_work = (int32_t)(sl.order + B);
+  sl.words = sl.cu_work + B + 1;
+  if (sl.words > kScheduleWords)
     return fail(WF_ERR_INVALID_ARG,
-                "schedule needs %lld words (batch %lld, %lld tokens); the allocation-free entry "
-                "point holds at most %lld: 3 * (batch + 1) + 2 * (ceil(nTokens / %d) + batch) "
-                "+ 8 <= %lld",
-                (long long)sl.words, (long long)B, (long long)tq, (long long)kScheduleWords,
-                kern.unit_rows, (long long)kScheduleWords);
+                "schedule needs %lld words (batch %lld); the allocation-free entry point holds "
+                "at most %lld: 4 * batch + 5 <= %lld, i.e. batch <= %lld",
+                (long long)sl.words, (long long)B, (long long)kScheduleWords,
+                (long long)kScheduleWords, (long long)((kScheduleWords - 5) / 4));
 
   DeviceState *ds = current_device_state(&st);
   if (!ds) return st;
@@ -171,8 +170,7 @@ extern "C" wf_status_t wf_attn_fwd_varlen_noalloc(
   p.sl = sl;
   cudaError_t e = launch_sched_prep(static_cast<const int32_t *>(qSeqLen->data),
                                     static_cast<const int32_t *>(kvSeqLen->data), (int32_t)B, tq,
-                                    tk, maskType == WF_MASK_CAUSAL ? 1 : 0, kern.unit_rows, ws, sl,
-                                    ds->status, cs);
+                                    tk, headNum, kern.unit_rows, ws, sl, ds->status, cs);
   if (e != cudaSuccess) return cuda_fail(e, "sched_prep launch");
   e = kern.launch(p, ds->sm_count, cs);
   if (e != cudaSuccess) return cuda_fail(e, "attention kernel launch");

@@ -388,14 +388,13 @@ wf_status_t wf_attn_fwd_debug(const wf_tensor_t *q, const wf_tensor_t *qRope, co
   size_t sched_bytes = 0;
   if (d.varlen) {
     const int64_t B = d.batch;
-    const int64_t cap = (d.tq + kern.unit_rows - 1) / kern.unit_rows + B;
-    if (cap * headNum > INT32_MAX) return fail(WF_ERR_UNSUPPORTED, "too many tiles");
+    const int64_t max_items = ((d.tq + kern.unit_rows - 1) / kern.unit_rows + B) * headNum;
+    if (max_items > INT32_MAX) return fail(WF_ERR_UNSUPPORTED, "too many work items");
     sl.cu_q = 2;
     sl.cu_k = (int32_t)(sl.cu_q + B + 1);
-    sl.cu_t = (int32_t)(sl.cu_k + B + 1);
-    sl.entries = (int32_t)(((sl.cu_t + B + 1) + 3) & ~int64_t(3));
-    sl.capacity = (int32_t)cap;
-    sl.words = sl.entries + 2 * cap;
+    sl.order = (int32_t)(sl.cu_k + B + 1);
+    sl.cu_work = (int32_t)(sl.order + B);
+    sl.words = sl.cu_work + B + 1;
     sched_bytes = ((size_t)sl.words * 4 + 255) & ~size_t(255);
   }
   const int64_t vt_ld = (n_keys + 3) & ~int64_t(3);
@@ -439,8 +438,8 @@ wf_status_t wf_attn_fwd_debug(const wf_tensor_t *q, const wf_tensor_t *qRope, co
     const int64_t B = d.batch;
     cudaError_t e = launch_sched_prep(static_cast<const int32_t *>(qSeqLen->data),
                                       static_cast<const int32_t *>(kvSeqLen->data), (int32_t)B,
-                                      d.tq, d.tk, maskType == WF_MASK_CAUSAL ? 1 : 0,
-                                      kern.unit_rows, ws, sl, ds->status, cs);
+                                      d.tq, d.tk, headNum, kern.unit_rows, ws, sl, ds->status,
+                                      cs);
     if (e != cudaSuccess) return cuda_fail(e, "sched_prep launch");
     p.ws = ws;
     p.sl = sl;

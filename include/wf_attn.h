@@ -167,9 +167,8 @@ wf_status_t wf_attn_fwd_debug(const wf_tensor_t *q, const wf_tensor_t *qRope,
  * CAUSAL; all tensors WF_BF16).  Instead of an allocated workspace, the
  * schedule tables live in a fixed array inside the library: 65536 int32
  * words (256 KiB) on every GPU that loads the library, held until the
- * process exits.  A call needs 3 * (batch + 1) + 2 * (ceil(nTokens / 256) +
- * batch) + 8 words; larger calls return WF_ERR_INVALID_ARG and launch
- * nothing.  The first call on a device looks the array's address up
+ * process exits.  A call needs 4 * batch + 5 words (batch <= 16382); larger
+ * calls return WF_ERR_INVALID_ARG and launch nothing.  The first call on a device looks the array's address up
  * (cudaGetSymbolAddress); make that first call before any stream capture.
  * All calls share the array: calls whose work overlaps on the GPU (e.g. on
  * different streams) race; calls in order on one stream do not, as each
