@@ -63,9 +63,10 @@ struct PPCfg {
   static constexpr uint32_t kIdescS = instr_desc(1, kBlockM, kBlockN, 0);
   static constexpr uint32_t kIdescPV = instr_desc(1, kBlockM, kNPV, 1);
   static constexpr uint32_t kTmemCols = 512;
-  // FMA-pipe exp2 share (of 16 columns): pays off where the QK product is 128
-  // wide; the 192-wide MLA product leaves the softmax enough time as it is.
-  static constexpr int kEmuPer16 = (DQK + DROPE) <= 128 ? 4 : 0;
+  // FMA-pipe exp2 share (of 16 columns).  Measured on B200 with waits that
+  // suspend instead of spinning, a share of 4/16 cost ~4% at head size 128
+  // and more with the 192-wide MLA product, so the MUFU unit does all of them.
+  static constexpr int kEmuPer16 = 0;
   static_assert(kKStages >= 1 && kVStages >= 1 && kSmemUsed <= 227 * 1024, "smem");
   static_assert(DQK % kKStep == 0 && DV % 32 == 0 && kNPV <= 128, "head dims");
 };
@@ -164,27 +165,39 @@ __device__ void pp_producer(const AttnParams &p, uint8_t *smem, PPCtrl *ctl, Pro
 }
 
 // ----------------------------------------------------------------------- MMA
-template <typename Cfg>
-__device__ __forceinline__ void pp_issue_s(uint32_t tmem, uint32_t qbase, uint32_t kbase,
-                                           int s) {
-#pragma unroll
-  for (int ks = 0; ks < Cfg::kSKStepsQK + Cfg::kSKStepsR; ++ks) {
-    const int atom = ks < Cfg::kSKStepsQK ? ks / 4 : Cfg::kQAtoms + (ks - Cfg::kSKStepsQK) / 4;
-    const int within = (ks < Cfg::kSKStepsQK ? ks % 4 : (ks - Cfg::kSKStepsQK) % 4) * 32;
-    const uint32_t off = atom * Cfg::kAtomBytes + within;
-    mma_f16_ss(tmem + (s ? 128u : 0u), smem_desc_sw128(qbase + off, 16, 1024),
-               smem_desc_sw128(kbase + off, 16, 1024), Cfg::kIdescS, ks > 0 ? 1u : 0u);
+// S = Q K^T: k-steps 0..KS, unrolled at compile time; q / k are the tile
+// descriptors, each k-step moves both by the same compile-time offset.
+template <typename Cfg, int KS>
+struct IssueS {
+  static __device__ __forceinline__ void run(uint32_t d, Desc q, Desc k) {
+    if constexpr (KS > 0) IssueS<Cfg, KS - 1>::run(d, q, k);
+    constexpr bool rope = KS >= Cfg::kSKStepsQK;
+    constexpr int atom = rope ? Cfg::kQAtoms + (KS - Cfg::kSKStepsQK) / 4 : KS / 4;
+    constexpr int within = (rope ? (KS - Cfg::kSKStepsQK) % 4 : KS % 4) * 32;
+    constexpr int off = (atom * Cfg::kAtomBytes + within) >> 4;
+    mma_f16_ss_at<off, off>(d, q, k, Cfg::kIdescS, KS > 0 ? 1u : 0u);
   }
+};
+// O (+)= P V: P read from TMEM (8 columns per k-step), V MN-major (16 rows of
+// 128 bytes per k-step).
+template <typename Cfg, int KS>
+struct IssuePV {
+  static __device__ __forceinline__ void run(uint32_t d, uint32_t p_tmem, Desc v, uint32_t acc0) {
+    if constexpr (KS > 0) IssuePV<Cfg, KS - 1>::run(d, p_tmem, v, acc0);
+    mma_f16_ts_at<KS * 8, ((KS * Cfg::kKStep * 128) >> 4)>(d, p_tmem, v, Cfg::kIdescPV,
+                                                         KS > 0 ? 1u : acc0);
+  }
+};
+
+template <typename Cfg>
+__device__ __forceinline__ void pp_issue_s(uint32_t tmem, Desc q, Desc k, int s) {
+  IssueS<Cfg, Cfg::kSKStepsQK + Cfg::kSKStepsR - 1>::run(tmem + (s ? 128u : 0u), q, k);
 }
 
 template <typename Cfg>
-__device__ __forceinline__ void pp_issue_pv(uint32_t tmem, uint32_t vbase, int s, bool accumulate) {
-#pragma unroll
-  for (int ks = 0; ks < Cfg::kPVKSteps; ++ks) {
-    const uint64_t bdesc = smem_desc_sw128(vbase + ks * Cfg::kKStep * 128, Cfg::kAtomBytes, 1024);
-    mma_f16_ts(tmem + (s ? 384u : 256u), tmem + (s ? 128u : 0u) + ks * 8, bdesc, Cfg::kIdescPV,
-               (accumulate || ks > 0) ? 1u : 0u);
-  }
+__device__ __forceinline__ void pp_issue_pv(uint32_t tmem, Desc v, int s, bool accumulate) {
+  IssuePV<Cfg, Cfg::kPVKSteps - 1>::run(tmem + (s ? 384u : 256u), tmem + (s ? 128u : 0u), v,
+                                        accumulate ? 1u : 0u);
 }
 
 template <typename Cfg>
@@ -194,9 +207,18 @@ __device__ void pp_mma(const AttnParams &p, uint8_t *smem, PPCtrl *ctl, uint32_t
   uint32_t cp[2] = {0, 0};    // PVs issued per tile slot (p_full completions consumed)
   uint32_t co[2] = {0, 0};    // units in which each tile slot took part (o_empty phases)
   bool ok = true;
-  const uint32_t qb[2] = {smem_u32(smem), smem_u32(smem + Cfg::kQTileBytes)};
-  auto kbase = [&](uint32_t gg) { return smem_u32(smem + Cfg::kKOff + (gg % Cfg::kKStages) * Cfg::kKBytes); };
-  auto vbase = [&](uint32_t gg) { return smem_u32(smem + Cfg::kVOff + (gg % Cfg::kVStages) * Cfg::kVBytes); };
+  // descriptor bases, computed once: Q tiles, and stage 0 of the K / V rings
+  // (stage i adds i * bytes-per-stage >> 4 to the low word)
+  const Desc qb[2] = {desc_split(smem_desc_sw128(smem_u32(smem), 16, 1024)),
+                      desc_split(smem_desc_sw128(smem_u32(smem + Cfg::kQTileBytes), 16, 1024))};
+  const Desc k0 = desc_split(smem_desc_sw128(smem_u32(smem + Cfg::kKOff), 16, 1024));
+  const Desc v0 = desc_split(smem_desc_sw128(smem_u32(smem + Cfg::kVOff), Cfg::kAtomBytes, 1024));
+  auto kbase = [&](uint32_t gg) {
+    return Desc{k0.lo + (gg % Cfg::kKStages) * (Cfg::kKBytes >> 4), k0.hi};
+  };
+  auto vbase = [&](uint32_t gg) {
+    return Desc{v0.lo + (gg % Cfg::kVStages) * (Cfg::kVBytes >> 4), v0.hi};
+  };
   auto wait_k = [&](uint32_t gg) {
     return bwait(&ctl->k_full[gg % Cfg::kKStages], (gg / Cfg::kKStages) & 1, &ctl->abort, p);
   };

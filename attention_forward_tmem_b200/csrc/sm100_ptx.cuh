@@ -32,15 +32,18 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
                "r"(bytes)
                : "memory");
 }
-// True once the phase with the given parity has completed.
+// True once the phase with the given parity has completed.  If it has not,
+// the thread is suspended until it completes or `kSuspendNs` elapse (so a
+// waiting warp does not spin and take issue slots from its neighbours).
+constexpr uint32_t kSuspendNs = 10000000;
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs)
       : "memory");
   return ok != 0;
 }
@@ -141,6 +144,44 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   d |= static_cast<uint64_t>(1) << 46;   // descriptor version (sm_100)
   d |= static_cast<uint64_t>(2) << 61;   // SWIZZLE_128B
   return d;
+}
+
+// Low / high 32-bit words of a descriptor; the start address lives in the
+// low 14 bits of the low word, so moving the start by `bytes` within the
+// 256 KB shared window is a 32-bit add of bytes >> 4 to the low word.
+struct Desc {
+  uint32_t lo, hi;
+};
+__device__ __forceinline__ Desc desc_split(uint64_t d) {
+  return {static_cast<uint32_t>(d), static_cast<uint32_t>(d >> 32)};
+}
+
+// One kind::f16 MMA (K = 16) with both operands in shared memory; the
+// descriptors are the precomputed bases `a`, `b` moved by the compile-time
+// offsets AOFF / BOFF (16-byte units).  D (+)= A * B.
+template <int AOFF, int BOFF>
+__device__ __forceinline__ void mma_f16_ss_at(uint32_t d_tmem, Desc a, Desc b, uint32_t idesc,
+                                              uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t.reg .b32 ta, tb;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\tadd.u32 ta, %1, %6;\n\tadd.u32 tb, %3, %7;\n\t"
+      "mov.b64 da, {ta, %2};\n\tmov.b64 db, {tb, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %8, p;\n\t}" ::"r"(d_tmem),
+      "r"(a.lo), "r"(a.hi), "r"(b.lo), "r"(b.hi), "r"(accumulate), "n"(AOFF), "n"(BOFF), "r"(idesc)
+      : "memory");
+}
+// One kind::f16 MMA (K = 16) with A in tensor memory at a_tmem + ATMEM columns
+// and B the precomputed base `b` moved by BOFF (16-byte units).
+template <int ATMEM, int BOFF>
+__device__ __forceinline__ void mma_f16_ts_at(uint32_t d_tmem, uint32_t a_tmem, Desc b,
+                                              uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t.reg .b32 ta, tb;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\tadd.u32 ta, %1, %5;\n\tadd.u32 tb, %2, %6;\n\t"
+      "mov.b64 db, {tb, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %7, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "r"(b.lo), "r"(b.hi), "r"(accumulate), "n"(ATMEM), "n"(BOFF), "r"(idesc)
+      : "memory");
 }
 
 // Instruction descriptor for kind::f16 / kind::tf32 with fp32 accumulation.
