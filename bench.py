@@ -371,7 +371,8 @@ def main():
                 "traffic": profiled_traffic(args.workload),
                 "peak_source": f"{peak_kind} bf16 burst (MEASURED_PEAKS.json)"
                 if peak_kind == "measured" else "fallback 1.59 PFLOP/s",
-                "kernel": "wf::attn_fwd_kernel", "algorithmic_flops_per_launch": wl.flops}
+                "kernel": "wf::attn_fwd_pp_kernel" if wl.w.dtype == torch.bfloat16 else "wf::attn_fwd_kernel",
+                "algorithmic_flops_per_launch": wl.flops}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload != "mla_varlen_prefill":
