@@ -232,6 +232,11 @@ wf_status_t wf_attn_fwd_debug(const wf_tensor_t *q, const wf_tensor_t *qRope, co
 
   Dims d{};
   d.varlen = qSeqLen != nullptr;
+  // The TF32 path reads V^T with the key index as the innermost TMA
+  // coordinate; a packed sequence may start at any token, which breaks the
+  // 16-byte rule on that coordinate, so fp32 is dense-only.
+  if (d.varlen && dt == WF_F32)
+    return fail(WF_ERR_UNSUPPORTED, "WF_F32 inputs are supported in the dense layout only");
   const int nd = d.varlen ? 3 : 4;
   if ((st = check_tensor(q, "q", nd, dt, true)) != WF_OK) return st;
   if ((st = check_tensor(k, "k", nd, dt, true)) != WF_OK) return st;

@@ -116,7 +116,8 @@ typedef struct wf_tensor {
  *   headNum % kvHeadNum == 0; query head h reads kv head h / (headNum/kvHeadNum).
  *   qkScale multiplies Q*K^T before the mask is added ([P2] row qkScale).
  *   dtypes: q, k, v, qRope, kRope, out all WF_BF16, or all WF_F32 (the F32
- *     path multiplies on TF32 tensor cores).  Dqk, Dv in {64, 96, 128};
+ *     path multiplies on TF32 tensor cores; dense layout only, packed F32
+ *     returns WF_ERR_UNSUPPORTED).  Dqk, Dv in {64, 96, 128};
  *     with rope: Dqk = 128, Dv = 128, BF16.
  *   Alignment: every data pointer 16-byte aligned; every stride except the
  *     last a multiple of 16 bytes.

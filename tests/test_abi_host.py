@@ -90,6 +90,7 @@ def test_valid_call_reaches_device_check(lib):
     ("mask_missing", L.WF_ERR_INVALID_ARG),
     ("mask_with_causal", L.WF_ERR_INVALID_ARG),
     ("mask_with_varlen", L.WF_ERR_UNSUPPORTED),
+    ("f32_varlen", L.WF_ERR_UNSUPPORTED),
     ("mask_bad_shape", L.WF_ERR_INVALID_ARG),
     ("mask_bad_dtype", L.WF_ERR_INVALID_ARG),
     ("rope_one_side", L.WF_ERR_INVALID_ARG),
@@ -127,6 +128,10 @@ def test_argument_errors(lib, case, expect):
         q, k, v, o = _t([300, 8, 128]), _t([300, 2, 128]), _t([300, 2, 128]), _t([300, 8, 128])
         kw.update(ql=_t([3], L.WF_I32), kl=_t([3], L.WF_I32), mask=_t([1, 1, 300, 300], L.WF_U8),
                   mt=L.WF_MASK_BOOL_KEEP)
+    elif case == "f32_varlen":
+        f = L.WF_F32
+        q, k, v, o = _t([300, 8, 128], f), _t([300, 2, 128], f), _t([300, 2, 128], f), _t([300, 8, 128], f)
+        kw.update(ql=_t([3], L.WF_I32), kl=_t([3], L.WF_I32))
     elif case == "mask_bad_shape":
         kw.update(mt=L.WF_MASK_BOOL_KEEP, mask=_t([2, 3, 100, 120], L.WF_U8))
     elif case == "mask_bad_dtype":
