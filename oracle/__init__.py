@@ -10,5 +10,7 @@ Contents:
   * ``sdpa`` / ``sdpa_rows``  -- ctypes front end of ``sdpa_oracle.c`` (fp64, OpenMP)
   * ``brute``                 -- pure-Python per-element loops for tiny inputs
   * ``kvcache_model``         -- plain Python model of the BlockKVCache contract
+  * ``merge``                 -- fp64 merge of results over disjoint key sets (by LSE)
 """
 from .sdpa import sdpa, sdpa_rows, build_oracle, oracle_threads, MASK_KINDS  # noqa: F401
+from .merge import merge, MERGE_PLANTS  # noqa: F401

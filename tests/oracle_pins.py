@@ -273,6 +273,68 @@ PINS = [pin_page_example_shape, pin_torch_no_mask, pin_torch_gqa, pin_torch_keep
         pin_torch_mla_concat, pin_brute_dense, pin_brute_packed, pin_uniform_closed_form,
         pin_mask_invariants, pin_fully_masked_rows, pin_lse]
 
+# ------------------------------------------------------------- merge pins
+# Each takes ``plant`` = a key of oracle.MERGE_PLANTS (0 = faithful merge).
+
+def _torch_lse(q, k, scale, mask=None):
+    group = q.shape[1] // k.shape[1]
+    s = q @ k.repeat_interleave(group, dim=1).transpose(-1, -2) * scale
+    if mask is not None:
+        s = s.masked_fill(~mask, -math.inf)
+    return torch.logsumexp(s, dim=-1)
+
+
+def pin_merge_random_key_sets(plant=0):
+    """Keys dealt at random into three disjoint sets (keep-masks); merging the
+    three partial results gives torch's attention and logsumexp over all keys."""
+    g = _rng(40)
+    q, k, v = _randn(g, 2, 4, 9, 8), _randn(g, 2, 2, 13, 8), _randn(g, 2, 2, 13, 5)
+    owner = torch.randint(0, 3, (13,), generator=g)
+    outs, lses = [], []
+    for s_ in range(3):
+        keep = (owner == s_).view(1, 1, 1, 13).expand(2, 4, 9, 13).to(torch.uint8)
+        o, l = oracle.sdpa(q, k, v, mask=keep, mask_kind="keep", qk_scale=0.3, with_lse=True)
+        outs.append(o)
+        lses.append(l)
+    out, lse = oracle.merge(np.stack(outs), np.stack(lses), plant=plant)
+    return _close(out, _torch_ref(q, k, v, 0.3).numpy()) and _close(lse, _torch_lse(q, k, 0.3).numpy())
+
+
+def pin_merge_causal_halves(plant=0):
+    """Causal rows split at key 5: rows 0..4 have nothing in the second half
+    (lse -inf, weight 0); the merge equals torch's causal attention."""
+    g = _rng(41)
+    q, k, v = _randn(g, 1, 2, 10, 8), _randn(g, 1, 2, 10, 8), _randn(g, 1, 2, 10, 6)
+    tril = torch.ones(10, 10, dtype=torch.bool).tril()
+    j = torch.arange(10)
+    outs, lses = [], []
+    for half in (j < 5, j >= 5):
+        keep = (tril & half.view(1, 10)).view(1, 1, 10, 10).expand(1, 2, 10, 10).to(torch.uint8)
+        o, l = oracle.sdpa(q, k, v, mask=keep, mask_kind="keep", qk_scale=0.5, with_lse=True)
+        outs.append(o)
+        lses.append(l)
+    ok = bool(np.all(lses[1][0, :, :5] == -np.inf))
+    out, lse = oracle.merge(np.stack(outs), np.stack(lses), plant=plant)
+    ref = _torch_ref(q, k, v, 0.5, mask=tril).numpy()
+    return ok and _close(out, ref) and _close(lse, _torch_lse(q, k, 0.5, tril).numpy())
+
+
+def pin_merge_closed_forms(plant=0):
+    """Equal lse: the mean of the parts and lse + ln 2.  One part at -inf: the
+    other part unchanged.  All parts at -inf: zero and -inf."""
+    a = np.array([[1.0, -2.0, 4.0]])
+    b = np.array([[3.0, 0.0, -4.0]])
+    out, lse = oracle.merge(np.stack([a, b]), np.array([[0.7], [0.7]]), plant=plant)
+    ok = _close(out, (a + b) / 2) and _close(lse, [0.7 + math.log(2.0)])
+    out, lse = oracle.merge(np.stack([a, b]), np.array([[-np.inf], [1.5]]), plant=plant)
+    ok &= _close(out, b) and _close(lse, [1.5])
+    out, lse = oracle.merge(np.stack([a, b]), np.array([[-np.inf], [-np.inf]]), plant=plant)
+    ok &= bool(np.all(out == 0.0)) and lse[0] == -np.inf
+    return ok
+
+
+MERGE_PINS = [pin_merge_random_key_sets, pin_merge_causal_halves, pin_merge_closed_forms]
+
 # Planted mistakes compiled into copies of the oracle (ORACLE_PLANT=n).
 PLANTS = {
     1: "GQA group index h % kvHeadNum instead of h / (headNum / kvHeadNum)",

@@ -22,6 +22,17 @@ def test_planted_mistake_is_caught(plant):
     assert failed, f"no pin catches planted mistake {plant}: {P.PLANTS[plant]}"
 
 
+@pytest.mark.parametrize("pin", P.MERGE_PINS, ids=lambda f: f.__name__)
+def test_merge_pin_holds(pin):
+    assert pin(0)
+
+
+@pytest.mark.parametrize("plant", sorted(oracle.MERGE_PLANTS), ids=lambda n: oracle.MERGE_PLANTS[n])
+def test_merge_planted_mistake_is_caught(plant):
+    failed = [p.__name__ for p in P.MERGE_PINS if not p(plant)]
+    assert failed, f"no pin catches planted merge mistake {plant}: {oracle.MERGE_PLANTS[plant]}"
+
+
 def test_rows_mode_matches_full():
     g = torch.Generator().manual_seed(30)
     lens = torch.tensor([7, 3, 9], dtype=torch.int32)
