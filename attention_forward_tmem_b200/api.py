@@ -81,15 +81,21 @@ def _require_cuda(*ts):
 
 def attn_fwd(q, k, v, *, qrope=None, krope=None, q_seqlen=None, kv_seqlen=None, mask=None,
              mask_type=None, head_num=None, kv_head_num=None, qk_scale=None, out=None,
-             stream=None, debug_flags=0, timeout_cycles=0):
+             return_lse=False, lse=None, num_splits=None, stream=None, debug_flags=0,
+             timeout_cycles=0):
     """out = softmax(q k^T * qk_scale + mask) v, see ``include/wf_attn.h``.
 
     Dense: q [B,Hq,Lq,D], k/v [B,Hkv,Lk,D].  Packed: q [T,Hq,D], k/v [Tk,Hkv,D]
     with int32 ``q_seqlen`` / ``kv_seqlen`` on the device.  ``mask_type``
     defaults to BOOL_KEEP for a bool mask, ADDITIVE for a float mask, NONE
     otherwise.  ``qk_scale`` defaults to 1/sqrt(Dqk + Drope).
+
+    ``return_lse`` (or a given fp32 ``lse`` tensor of out's shape without the
+    last dim) also returns the natural-log LSE of every row: ``(out, lse)``.
+    ``num_splits``: None/0 automatic split-KV, 1 none, n > 1 forced
+    (``wf_attn_fwd_ex``).
     """
-    _require_cuda(q, k, v, qrope, krope, q_seqlen, kv_seqlen, mask, out)
+    _require_cuda(q, k, v, qrope, krope, q_seqlen, kv_seqlen, mask, out, lse)
     varlen = q_seqlen is not None
     if head_num is None:
         head_num = q.shape[1]
@@ -111,11 +117,21 @@ def attn_fwd(q, k, v, *, qrope=None, krope=None, q_seqlen=None, kv_seqlen=None, 
     if mask is not None:
         while mask.dim() < 4:
             mask = mask.unsqueeze(0)
+    want_lse = return_lse or lse is not None
+    if want_lse and lse is None:
+        lse = torch.empty(out.shape[:-1], dtype=torch.float32, device=q.device)
     descs = [describe(x) for x in (q, qrope, k, krope, v, q_seqlen, kv_seqlen, mask)]
     od = describe(out)
     lib = L.load()
     with torch.cuda.device(q.device):
-        if debug_flags or timeout_cycles:
+        if want_lse or num_splits is not None:
+            if debug_flags or timeout_cycles:
+                raise ValueError("debug switches do not combine with lse / num_splits")
+            ld = describe(lse) if want_lse else None
+            st = lib.wf_attn_fwd_ex(*[_ref(d) for d in descs], int(head_num), int(kv_head_num),
+                                    float(qk_scale), int(mask_type), ctypes.byref(od), _ref(ld),
+                                    int(num_splits or 0), _stream(stream))
+        elif debug_flags or timeout_cycles:
             st = lib.wf_attn_fwd_debug(*[_ref(d) for d in descs], int(head_num), int(kv_head_num),
                                        float(qk_scale), int(mask_type), ctypes.byref(od),
                                        _stream(stream), int(debug_flags), int(timeout_cycles))
@@ -123,7 +139,34 @@ def attn_fwd(q, k, v, *, qrope=None, krope=None, q_seqlen=None, kv_seqlen=None, 
             st = lib.wf_attn_fwd(*[_ref(d) for d in descs], int(head_num), int(kv_head_num),
                                  float(qk_scale), int(mask_type), ctypes.byref(od), _stream(stream))
     _check(st)
-    return out
+    return (out, lse) if want_lse else out
+
+
+def merge(out_parts, lse_parts, *, out=None, lse=None, stream=None):
+    """Combine results over disjoint key sets (``wf_attn_merge``).
+
+    ``out_parts`` [S, ..., Dv] (fp32 or bf16), ``lse_parts`` [S, ...] fp32
+    (natural log).  Returns ``(out, lse)``; ``out`` defaults to the parts'
+    dtype.  The row dims are flattened by views, so they must be viewable as
+    one dim.
+    """
+    _require_cuda(out_parts, lse_parts, out, lse)
+    S, dv = out_parts.shape[0], out_parts.shape[-1]
+    rows_shape = tuple(out_parts.shape[1:-1])
+    if tuple(lse_parts.shape) != (S,) + rows_shape:
+        raise ValueError(f"lse_parts {tuple(lse_parts.shape)} does not match out_parts {tuple(out_parts.shape)}")
+    if out is None:
+        out = torch.empty(rows_shape + (dv,), dtype=out_parts.dtype, device=out_parts.device)
+    if lse is None:
+        lse = torch.empty(rows_shape, dtype=torch.float32, device=out_parts.device)
+    pd = describe(out_parts.view(S, -1, dv))
+    ld = describe(lse_parts.view(S, -1))
+    od = describe(out.view(-1, dv))
+    ed = describe(lse.view(-1))
+    with torch.cuda.device(out_parts.device):
+        _check(L.load().wf_attn_merge(ctypes.byref(pd), ctypes.byref(ld), ctypes.byref(od),
+                                      ctypes.byref(ed), _stream(stream)))
+    return out, lse
 
 
 def device_status(stream=None) -> None:

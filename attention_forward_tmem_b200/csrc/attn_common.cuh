@@ -22,18 +22,28 @@
 namespace wf {
 
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 
 
 struct TileInfo {
   int32_t b, h, hk, q0, lq, lk, qrow, krow, n_kv, off, tma_b;
+  int32_t sp, kt0;     // split index, first KV tile of the split (0 without split)
 };
 
 // Sub-tile `sub` (128 rows each) of work item `t`; the enumeration order is
 // described in attn_params.h (per sequence, per kv head, longest unit first,
-// GQA heads adjacent).
+// GQA heads adjacent; with split-KV the splits of one unit are adjacent).
+// krow / n_kv describe the KV tiles this item visits: tiles [kt0, kt0 + n_kv)
+// of the sequence, krow being the TMA row of tile kt0.
 __device__ __forceinline__ TileInfo tile_info(const AttnParams &p, int32_t t, int32_t sub) {
   TileInfo ti;
+  ti.sp = 0;
+  ti.kt0 = 0;
+  if (p.n_split > 1) {
+    ti.sp = t % p.n_split;
+    t /= p.n_split;
+  }
   const int32_t G = p.group;
   const bool causal = p.mask_kind == kMaskCausal;
   int32_t r, n_units;
@@ -69,7 +79,8 @@ __device__ __forceinline__ TileInfo tile_info(const AttnParams &p, int32_t t, in
   const int32_t j = r / G;
   ti.h = ti.hk * G + (r - j * G);
   const int32_t u = causal ? n_units - 1 - j : j;
-  ti.q0 = u * p.unit_rows + sub * kBlockM;
+  const int32_t u0 = u * p.unit_rows;
+  ti.q0 = u0 + sub * kBlockM;
   ti.qrow = (p.varlen ? __ldg(p.ws + p.sl.cu_q + ti.b) : 0) + ti.q0;
   ti.off = ti.lk - ti.lq;
   int32_t kend = ti.q0 < ti.lq ? ti.lk : 0;            // no valid row: nothing to do
@@ -78,12 +89,24 @@ __device__ __forceinline__ TileInfo tile_info(const AttnParams &p, int32_t t, in
     kend = min(kend, last + ti.off);
   }
   ti.n_kv = kend > 0 ? (kend + kBlockN - 1) / kBlockN : 0;
+  if (p.n_split > 1) {
+    // The split bounds come from the whole unit, so both sub-tiles of a unit
+    // visit the same KV tiles (the CTA loads each tile once for both).
+    int32_t uend = u0 < ti.lq ? ti.lk : 0;
+    if (causal) uend = min(uend, min(u0 + p.unit_rows, ti.lq) + ti.off);
+    const int32_t n_unit = uend > 0 ? (uend + kBlockN - 1) / kBlockN : 0;
+    const int32_t per = (n_unit + p.n_split - 1) / p.n_split;
+    const int32_t lo = min(ti.sp * per, n_unit);
+    ti.kt0 = lo;
+    ti.n_kv = max(min(lo + per, ti.n_kv) - lo, 0);
+    ti.krow += lo * kBlockN;
+  }
   return ti;
 }
 
 __device__ __forceinline__ int32_t num_units(const AttnParams &p) {
-  if (!p.varlen) return p.n_units_dense;
-  return __ldg(p.ws);
+  const int32_t base = p.varlen ? __ldg(p.ws) : p.n_units_dense;
+  return p.n_split > 1 ? base * p.n_split : base;
 }
 
 // Bounded wait.  Returns false (and raises the CTA abort flag) on expiry, or
@@ -253,13 +276,40 @@ __device__ __forceinline__ void store_row(const AttnParams &p, const TileInfo &t
   }
 }
 
+// Result of one row: O / l to out (and its LSE when asked for), or, with
+// split-KV, the partial row normalised over this split's keys plus its LSE to
+// the partial buffers.  LSE = ln sum_j exp(x_j) = (m + log2 l) ln 2, -inf for a
+// row that saw no key (l = 0, O = 0).
+template <typename T, int DV>
+__device__ __forceinline__ void store_result(const AttnParams &p, const TileInfo &ti, int32_t row,
+                                             const float (&o)[DV], float m, float l) {
+  const float inv = l > 0.f ? 1.f / l : 0.f;
+  const float lse = l > 0.f ? (m + __log2f(l)) * kLn2 : -INFINITY;
+  if (p.n_split > 1) {
+    const int64_t r = p.varlen ? (int64_t)(ti.qrow - ti.q0 + row) * p.hq + ti.h
+                               : ((int64_t)ti.b * p.hq + ti.h) * p.lq + row;
+    const int64_t idx = (int64_t)ti.sp * p.part_rows + r;
+    float *dst = p.part_o + idx * DV;
+#pragma unroll
+    for (int c = 0; c < DV; c += 4)
+      *reinterpret_cast<float4 *>(dst + c) =
+          make_float4(o[c] * inv, o[c + 1] * inv, o[c + 2] * inv, o[c + 3] * inv);
+    p.part_lse[idx] = lse;
+  } else {
+    store_row<T, DV>(p, ti, row, o, inv);
+    if (p.lse)
+      p.lse[(int64_t)ti.b * p.l_sb + (int64_t)ti.h * p.l_sh +
+            (int64_t)(p.varlen ? ti.qrow + (row - ti.q0) : row) * p.l_si] = lse;
+  }
+}
+
 template <typename T, int DV>
 __device__ __forceinline__ void store_zero_row(const AttnParams &p, const TileInfo &ti,
                                                int32_t row) {
   float z[DV];
 #pragma unroll
   for (int c = 0; c < DV; ++c) z[c] = 0.f;
-  store_row<T, DV>(p, ti, row, z, 0.f);
+  store_result<T, DV>(p, ti, row, z, -INFINITY, 0.f);
 }
 
 // Load DV fp32 columns of this thread's TMEM lane starting at `taddr`.

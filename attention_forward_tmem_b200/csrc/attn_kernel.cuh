@@ -264,7 +264,7 @@ __device__ void softmax_role(const AttnParams &p, AttnCtrl *ctl, uint32_t tmem) 
       uint32_t sr[128];
       tmem_ld_x128(tmem + lane_base + sb * 128, sr);
       float x[128];
-      const float alpha = softmax_row<0>(p, ti, row, j * kBlockN, sr, x, m, l);
+      const float alpha = softmax_row<0>(p, ti, row, (ti.kt0 + j) * kBlockN, sr, x, m, l);
       tmem_store_p<Cfg::kTF32>(tmem + lane_base + sb * 128, x);
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
         // O holds the sum up to tile j-1 once PV[gg-1] is done.
@@ -291,7 +291,7 @@ __device__ void softmax_role(const AttnParams &p, AttnCtrl *ctl, uint32_t tmem) 
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(&ctl->o_empty);
-    if (row_valid) store_row<T, DV>(p, ti, row, o, l > 0.f ? 1.f / l : 0.f);
+    if (row_valid) store_result<T, DV>(p, ti, row, o, m, l);
   }
 }
 

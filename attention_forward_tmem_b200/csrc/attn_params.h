@@ -53,6 +53,19 @@ struct alignas(64) AttnParams {
   int32_t n_units_dense, units_per_bh;           // dense: total units, units per (b, h)
   const int32_t *ws;                             // varlen schedule (device)
   SchedLayout sl;
+  // Split-KV: with n_split > 1 every unit's KV tiles are dealt into n_split
+  // contiguous ranges, one work item each (item = unit * n_split + split);
+  // each writes its rows normalised over its own keys, in fp32, to
+  // part_o [n_split][part_rows][DV] and their natural-log LSE to
+  // part_lse [n_split][part_rows], and a merge pass combines them.  Row index:
+  // dense ((b * hq + h) * lq + i), packed (token * hq + h).
+  int32_t n_split;
+  float *part_o, *part_lse;
+  int64_t part_rows;
+  // Optional natural-log LSE of every row (n_split <= 1 only; NULL = none),
+  // element strides (batch, head, row) as for out.
+  float *lse;
+  int64_t l_sb, l_sh, l_si;
   float scale_log2;                              // qkScale * log2(e)
   int32_t *status;                               // device status word
   long long timeout_cycles;
@@ -73,6 +86,28 @@ AttnKernel find_attn_kernel(int dtype, int dqk, int drope, int dv);
 cudaError_t launch_transpose_v(const float *v, int64_t s_row, int64_t s_head, int64_t s_batch,
                                int32_t rows, int32_t heads, int32_t batch, int32_t d, float *vt,
                                int64_t ld, cudaStream_t stream);
+
+// Merge of per-key-set partial results by their LSE (merge.cu).  Row r of
+// the output decomposes as r = (i0 * n1 + i1) * n2 + i2.
+struct MergeParams {
+  const void *parts;         // [n_split][rows][dv], element strides ss / sr
+  int32_t parts_bf16;        // 0: fp32, 1: bf16
+  int64_t p_ss, p_sr;
+  const float *lses;         // [n_split][rows], element strides
+  int64_t l_ss, l_sr;
+  int32_t n_split, dv;
+  int64_t rows, n1, n2;
+  const int32_t *sched;      // packed schedule words (or NULL): nothing is merged if
+  int32_t sched_tokens;      // the length check failed (word 1), and only rows below
+                             // sched[sched_tokens] * n2 (the sequences' tokens) are
+  void *out;
+  int32_t out_bf16;
+  int64_t o_s0, o_s1, o_s2;
+  float *lse;                // NULL: not wanted
+  int64_t e_s0, e_s1, e_s2;
+};
+
+cudaError_t launch_merge(const MergeParams &mp, cudaStream_t stream);
 
 cudaError_t launch_sched_prep(const int32_t *q_len, const int32_t *k_len, int32_t batch,
                               int64_t n_q_tokens, int64_t n_k_tokens, int32_t head_num,

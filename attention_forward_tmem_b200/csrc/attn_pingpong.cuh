@@ -314,7 +314,7 @@ __device__ void pp_softmax(const AttnParams &p, PPCtrl *ctl, uint32_t tmem, int 
       uint32_t sr[128];
       tmem_ld_x128(s_addr, sr);
       float x[128];
-      const float alpha = softmax_row<kEmuPer16>(p, ti, row, j * kBlockN, sr, x, m, l);
+      const float alpha = softmax_row<kEmuPer16>(p, ti, row, (ti.kt0 + j) * kBlockN, sr, x, m, l);
       tmem_store_p<false>(s_addr, x);
       // S_s(j) done implies PV_s(j-1) done: O_s may be rescaled right away.
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) tmem_scale_row<DV>(o_addr, alpha);
@@ -332,7 +332,7 @@ __device__ void pp_softmax(const AttnParams &p, PPCtrl *ctl, uint32_t tmem, int 
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(&ctl->o_empty[s]);
-    if (row_valid) store_row<T, DV>(p, ti, row, o, l > 0.f ? 1.f / l : 0.f);
+    if (row_valid) store_result<T, DV>(p, ti, row, o, m, l);
   }
 }
 

@@ -1,0 +1,102 @@
+// merge.cu -- combine attention results computed over disjoint key sets.
+//
+// The pages name the uses (context-parallel attention in "Core 注意力",
+// section "选择最窄的入口"; calcType RING in the "MLA Prefill" parameter
+// table) but not the step; it follows from the softmax definition.  For a row
+// whose keys were split into sets s = 1..S, each with its normalised result
+// out_s and natural-log LSE lse_s:
+//     lse = ln sum_s exp(lse_s),      out = sum_s exp(lse_s - lse) * out_s.
+// A set with lse_s = -inf (no visible key) has weight 0; a row with every
+// set at -inf is 0 with LSE -inf.  The largest lse_s is subtracted before
+// exponentiating.
+//
+// One warp per row, four consecutive columns per lane per pass (128 columns
+// a pass); HBM-bound: it reads S partial rows and writes one.
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "attn_params.h"
+#include "sm100_ptx.cuh"
+
+namespace wf {
+namespace {
+
+constexpr int kMergeWarps = 8;
+constexpr float kLog2eM = 1.4426950408889634f;
+constexpr float kLn2M = 0.6931471805599453f;
+
+__device__ __forceinline__ void load4(const void *base, int64_t idx, bool bf16, float (&v)[4]) {
+  if (bf16) {
+    const uint2 u = *reinterpret_cast<const uint2 *>(reinterpret_cast<const __nv_bfloat16 *>(base) + idx);
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+    v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+  } else {
+    const float4 f = *reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(base) + idx);
+    v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+  }
+}
+
+__device__ __forceinline__ void store4(void *base, int64_t idx, bool bf16, const float (&v)[4]) {
+  if (bf16) {
+    uint2 u;
+    u.x = pack_bf16x2(v[0], v[1]);
+    u.y = pack_bf16x2(v[2], v[3]);
+    *reinterpret_cast<uint2 *>(reinterpret_cast<__nv_bfloat16 *>(base) + idx) = u;
+  } else {
+    *reinterpret_cast<float4 *>(reinterpret_cast<float *>(base) + idx) = make_float4(v[0], v[1], v[2], v[3]);
+  }
+}
+
+__global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(const __grid_constant__ MergeParams mp) {
+  int64_t rows = mp.rows;
+  if (mp.sched) {
+    if (mp.sched[1] != 0) return;                                   // lengths were rejected
+    rows = min(rows, (int64_t)mp.sched[mp.sched_tokens] * mp.n2);   // rows of the sequences
+  }
+  const int64_t r = (int64_t)blockIdx.x * kMergeWarps + (threadIdx.x >> 5);
+  if (r >= rows) return;
+  const int lane = threadIdx.x & 31;
+  const int64_t i2 = r % mp.n2, i01 = r / mp.n2;
+  const int64_t i1 = i01 % mp.n1, i0 = i01 / mp.n1;
+
+  float top = -INFINITY;
+  for (int s = 0; s < mp.n_split; ++s) top = fmaxf(top, mp.lses[s * mp.l_ss + r * mp.l_sr]);
+  const bool empty = top == -INFINITY;
+  float total = 0.f;
+  if (!empty)
+    for (int s = 0; s < mp.n_split; ++s)
+      total += ex2_approx((mp.lses[s * mp.l_ss + r * mp.l_sr] - top) * kLog2eM);
+  const float inv = empty ? 0.f : 1.f / total;
+
+  const int64_t obase = i0 * mp.o_s0 + i1 * mp.o_s1 + i2 * mp.o_s2;
+  for (int c = lane * 4; c < mp.dv; c += 128) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    if (!empty) {
+      for (int s = 0; s < mp.n_split; ++s) {
+        const float ls = mp.lses[s * mp.l_ss + r * mp.l_sr];
+        if (ls == -INFINITY) continue;                 // weight 0 (its row may be anything)
+        const float w = ex2_approx((ls - top) * kLog2eM) * inv;
+        float v[4];
+        load4(mp.parts, s * mp.p_ss + r * mp.p_sr + c, mp.parts_bf16 != 0, v);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[e] = fmaf(w, v[e], acc[e]);
+      }
+    }
+    store4(mp.out, obase + c, mp.out_bf16 != 0, acc);
+  }
+  if (mp.lse && lane == 0)
+    mp.lse[i0 * mp.e_s0 + i1 * mp.e_s1 + i2 * mp.e_s2] = empty ? -INFINITY : top + __log2f(total) * kLn2M;
+}
+
+}  // namespace
+
+cudaError_t launch_merge(const MergeParams &mp, cudaStream_t stream) {
+  if (mp.rows <= 0) return cudaSuccess;
+  const int64_t blocks = (mp.rows + kMergeWarps - 1) / kMergeWarps;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  merge_kernel<<<static_cast<unsigned>(blocks), kMergeWarps * 32, 0, stream>>>(mp);
+  return cudaGetLastError();
+}
+
+}  // namespace wf

@@ -162,6 +162,7 @@ extern "C" wf_status_t wf_attn_fwd_varlen_noalloc(
   p.hkv = kvHeadNum;
   p.group = headNum / kvHeadNum;
   p.varlen = 1;
+  p.n_split = 1;
   p.unit_rows = kern.unit_rows;
   p.scale_log2 = qkScale * 1.4426950408889634f;
   p.status = ds->status;

@@ -6,6 +6,7 @@
 // headNum, qkScale, kvHeadNum, maskType, attenOut; every call returns a
 // status); dense [B, H, L, D] layout and mask meaning: "Core 注意力"
 // (WorldFoundry docs), example section.
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -187,6 +188,9 @@ wf_status_t check_tensor(const wf_tensor_t *t, const char *name, int ndim, int32
   return WF_OK;
 }
 
+constexpr int32_t kMaxSplits = 128;        // largest numSplits accepted
+constexpr int64_t kMinTilesPerSplit = 4;   // automatic split: KV tiles per split, at least
+
 struct Dims {
   bool varlen;
   int64_t batch, lq, lk, tq, tk, dqk, dv, drope;
@@ -198,13 +202,30 @@ using namespace wf;
 
 extern "C" {
 
+static wf_status_t attn_fwd_impl(const wf_tensor_t *q, const wf_tensor_t *qRope, const wf_tensor_t *k,
+                                 const wf_tensor_t *kRope, const wf_tensor_t *v,
+                                 const wf_tensor_t *qSeqLen, const wf_tensor_t *kvSeqLen,
+                                 const wf_tensor_t *mask, int32_t headNum, int32_t kvHeadNum,
+                                 float qkScale, int32_t maskType, wf_tensor_t *out, wf_tensor_t *lse,
+                                 int32_t numSplits, void *stream, uint32_t debug_flags,
+                                 int64_t timeout_cycles);
+
 wf_status_t wf_attn_fwd(const wf_tensor_t *q, const wf_tensor_t *qRope, const wf_tensor_t *k,
                         const wf_tensor_t *kRope, const wf_tensor_t *v, const wf_tensor_t *qSeqLen,
                         const wf_tensor_t *kvSeqLen, const wf_tensor_t *mask, int32_t headNum,
                         int32_t kvHeadNum, float qkScale, int32_t maskType, wf_tensor_t *out,
                         void *stream) {
-  return wf_attn_fwd_debug(q, qRope, k, kRope, v, qSeqLen, kvSeqLen, mask, headNum, kvHeadNum,
-                           qkScale, maskType, out, stream, 0u, 0);
+  return attn_fwd_impl(q, qRope, k, kRope, v, qSeqLen, kvSeqLen, mask, headNum, kvHeadNum, qkScale,
+                       maskType, out, nullptr, 0, stream, 0u, 0);
+}
+
+wf_status_t wf_attn_fwd_ex(const wf_tensor_t *q, const wf_tensor_t *qRope, const wf_tensor_t *k,
+                           const wf_tensor_t *kRope, const wf_tensor_t *v, const wf_tensor_t *qSeqLen,
+                           const wf_tensor_t *kvSeqLen, const wf_tensor_t *mask, int32_t headNum,
+                           int32_t kvHeadNum, float qkScale, int32_t maskType, wf_tensor_t *out,
+                           wf_tensor_t *lse, int32_t numSplits, void *stream) {
+  return attn_fwd_impl(q, qRope, k, kRope, v, qSeqLen, kvSeqLen, mask, headNum, kvHeadNum, qkScale,
+                       maskType, out, lse, numSplits, stream, 0u, 0);
 }
 
 wf_status_t wf_attn_fwd_debug(const wf_tensor_t *q, const wf_tensor_t *qRope, const wf_tensor_t *k,
@@ -213,6 +234,69 @@ wf_status_t wf_attn_fwd_debug(const wf_tensor_t *q, const wf_tensor_t *qRope, co
                               const wf_tensor_t *mask, int32_t headNum, int32_t kvHeadNum,
                               float qkScale, int32_t maskType, wf_tensor_t *out, void *stream,
                               uint32_t debug_flags, int64_t timeout_cycles) {
+  return attn_fwd_impl(q, qRope, k, kRope, v, qSeqLen, kvSeqLen, mask, headNum, kvHeadNum, qkScale,
+                       maskType, out, nullptr, 0, stream, debug_flags, timeout_cycles);
+}
+
+wf_status_t wf_attn_merge(const wf_tensor_t *outParts, const wf_tensor_t *lseParts, wf_tensor_t *out,
+                          wf_tensor_t *lse, void *stream) {
+  clear_error();
+  wf_status_t st;
+  if (!outParts || !lseParts || !out) return fail(WF_ERR_INVALID_ARG, "outParts, lseParts and out are required");
+  const int32_t pdt = outParts->dtype, odt = out->dtype;
+  if ((pdt != WF_F32 && pdt != WF_BF16) || (odt != WF_F32 && odt != WF_BF16))
+    return fail(WF_ERR_UNSUPPORTED, "outParts / out dtype must be WF_F32 or WF_BF16");
+  if ((st = check_tensor(outParts, "outParts", 3, pdt, true)) != WF_OK) return st;
+  if ((st = check_tensor(lseParts, "lseParts", 2, WF_F32, false)) != WF_OK) return st;
+  if ((st = check_tensor(out, "out", 2, odt, true)) != WF_OK) return st;
+  if (lse && (st = check_tensor(lse, "lse", 1, WF_F32, false)) != WF_OK) return st;
+  const int64_t S = outParts->shape[0], R = outParts->shape[1], dv = outParts->shape[2];
+  if (lseParts->shape[0] != S || lseParts->shape[1] != R)
+    return fail(WF_ERR_INVALID_ARG, "lseParts must be [%lld, %lld]", (long long)S, (long long)R);
+  if (out->shape[0] != R || out->shape[1] != dv)
+    return fail(WF_ERR_INVALID_ARG, "out must be [%lld, %lld]", (long long)R, (long long)dv);
+  if (lse && lse->shape[0] != R) return fail(WF_ERR_INVALID_ARG, "lse must be [%lld]", (long long)R);
+  if (dv % 4 != 0) return fail(WF_ERR_UNSUPPORTED, "head size %lld is not a multiple of 4", (long long)dv);
+  if (S < 1 && R > 0) return fail(WF_ERR_INVALID_ARG, "at least one part is needed");
+  if ((numel(lseParts) > 0 && reinterpret_cast<uintptr_t>(lseParts->data) % 4) ||
+      (lse && numel(lse) > 0 && reinterpret_cast<uintptr_t>(lse->data) % 4))
+    return fail(WF_ERR_INVALID_ARG, "lse tensors must be 4-byte aligned");
+  if (R == 0 || dv == 0) return WF_OK;
+  DeviceState *ds = current_device_state(&st);
+  if (!ds) return st;
+  MergeParams mp{};
+  mp.parts = outParts->data;
+  mp.parts_bf16 = pdt == WF_BF16;
+  mp.p_ss = outParts->stride[0];
+  mp.p_sr = outParts->stride[1];
+  mp.lses = static_cast<const float *>(lseParts->data);
+  mp.l_ss = lseParts->stride[0];
+  mp.l_sr = lseParts->stride[1];
+  mp.n_split = (int32_t)S;
+  mp.dv = (int32_t)dv;
+  mp.rows = R;
+  mp.n1 = 1;
+  mp.n2 = R;
+  mp.out = out->data;
+  mp.out_bf16 = odt == WF_BF16;
+  mp.o_s2 = out->stride[0];
+  if (lse) {
+    mp.lse = static_cast<float *>(lse->data);
+    mp.e_s2 = lse->stride[0];
+  }
+  cudaError_t e = launch_merge(mp, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+  return WF_OK;
+}
+
+// The forward behind every attention entry point.
+static wf_status_t attn_fwd_impl(const wf_tensor_t *q, const wf_tensor_t *qRope, const wf_tensor_t *k,
+                                 const wf_tensor_t *kRope, const wf_tensor_t *v,
+                                 const wf_tensor_t *qSeqLen, const wf_tensor_t *kvSeqLen,
+                                 const wf_tensor_t *mask, int32_t headNum, int32_t kvHeadNum,
+                                 float qkScale, int32_t maskType, wf_tensor_t *out, wf_tensor_t *lse,
+                                 int32_t numSplits, void *stream, uint32_t debug_flags,
+                                 int64_t timeout_cycles) {
   clear_error();
   wf_status_t st;
   if (!q || !k || !v || !out) return fail(WF_ERR_INVALID_ARG, "q, k, v and out are required");
@@ -283,6 +367,18 @@ wf_status_t wf_attn_fwd_debug(const wf_tensor_t *q, const wf_tensor_t *qRope, co
       if (kRope->shape[i] != k->shape[i]) return fail(WF_ERR_INVALID_ARG, "kRope shape does not match k");
     }
   }
+
+  // lse: out's shape without the head-size dim, fp32, any strides
+  if (lse) {
+    if ((st = check_tensor(lse, "lse", nd - 1, WF_F32, false)) != WF_OK) return st;
+    for (int i = 0; i < nd - 1; ++i)
+      if (lse->shape[i] != out->shape[i])
+        return fail(WF_ERR_INVALID_ARG, "lse must have out's shape without its last dim");
+    if (numel(lse) > 0 && reinterpret_cast<uintptr_t>(lse->data) % 4)
+      return fail(WF_ERR_INVALID_ARG, "lse: data not 4-byte aligned");
+  }
+  if (numSplits < 0 || numSplits > kMaxSplits)
+    return fail(WF_ERR_INVALID_ARG, "numSplits %d: 0 (automatic) or 1..%d", numSplits, kMaxSplits);
 
   // mask
   const bool explicit_mask = maskType == WF_MASK_BOOL_KEEP || maskType == WF_MASK_ADDITIVE;
@@ -371,6 +467,12 @@ wf_status_t wf_attn_fwd_debug(const wf_tensor_t *q, const wf_tensor_t *qRope, co
     p.o_sh = out->stride[1];
     p.o_si = out->stride[0];
   }
+  if (lse) {
+    p.lse = static_cast<float *>(lse->data);
+    p.l_sb = d.varlen ? 0 : lse->stride[0];
+    p.l_sh = lse->stride[1];
+    p.l_si = d.varlen ? lse->stride[0] : lse->stride[2];
+  }
   p.mask = explicit_mask ? mask->data : nullptr;
   p.m_sb = ms[0];
   p.m_sh = ms[1];
@@ -388,12 +490,25 @@ wf_status_t wf_attn_fwd_debug(const wf_tensor_t *q, const wf_tensor_t *qRope, co
   p.timeout_cycles = timeout_cycles > 0 ? timeout_cycles : (2LL << 30);
   p.debug_flags = debug_flags;
 
-  // Per-stream workspace: [schedule tables (varlen)] [V^T (fp32)], 256-byte aligned parts.
+  // Split-KV: automatic only in the dense layout (the packed unit count is
+  // known on the device alone), when the units cannot fill the SMs: as many
+  // splits as fill them, each with at least kMinTilesPerSplit KV tiles.
+  const int64_t dense_units = d.varlen ? 0 : ((d.lq + kern.unit_rows - 1) / kern.unit_rows) * d.batch * headNum;
+  int32_t n_split = numSplits > 0 ? numSplits : 1;
+  if (numSplits == 0 && !d.varlen && n_keys > 0 && dense_units > 0 && dense_units < ds->sm_count) {
+    const int64_t by_grid = ds->sm_count / dense_units;
+    const int64_t by_len = ((d.lk + kBlockN - 1) / kBlockN) / kMinTilesPerSplit;
+    n_split = (int32_t)std::max<int64_t>(1, std::min(by_grid, by_len));
+  }
+  p.n_split = n_split;
+
+  // Per-stream workspace: [schedule tables (varlen)] [V^T (fp32)] [split
+  // partials: out fp32, lse fp32], 256-byte aligned parts.
   SchedLayout sl{};
   size_t sched_bytes = 0;
   if (d.varlen) {
     const int64_t B = d.batch;
-    const int64_t max_items = ((d.tq + kern.unit_rows - 1) / kern.unit_rows + B) * headNum;
+    const int64_t max_items = ((d.tq + kern.unit_rows - 1) / kern.unit_rows + B) * headNum * n_split;
     if (max_items > INT32_MAX) return fail(WF_ERR_UNSUPPORTED, "too many work items");
     sl.cu_q = 2;
     sl.cu_k = (int32_t)(sl.cu_q + B + 1);
@@ -404,11 +519,20 @@ wf_status_t wf_attn_fwd_debug(const wf_tensor_t *q, const wf_tensor_t *qRope, co
   }
   const int64_t vt_ld = (n_keys + 3) & ~int64_t(3);
   const int64_t vt_batch = d.varlen ? 1 : d.batch;
-  const size_t vt_bytes = dt == WF_F32 ? (size_t)(vt_batch * kvHeadNum * d.dv * vt_ld) * 4 : 0;
+  const size_t vt_bytes =
+      dt == WF_F32 ? ((size_t)(vt_batch * kvHeadNum * d.dv * vt_ld) * 4 + 255) & ~size_t(255) : 0;
+  const int64_t part_rows = n_split > 1 ? (d.varlen ? d.tq : d.batch * d.lq) * headNum : 0;
+  const size_t part_o_bytes = ((size_t)n_split * part_rows * d.dv * 4 + 255) & ~size_t(255);
+  const size_t part_l_bytes = ((size_t)n_split * part_rows * 4 + 255) & ~size_t(255);
+  const size_t ws_bytes = sched_bytes + vt_bytes + part_o_bytes + part_l_bytes;
   int32_t *ws = nullptr;
-  if (sched_bytes + vt_bytes > 0 &&
-      (st = stream_workspace(dev, cs, sched_bytes + vt_bytes, &ws)) != WF_OK)
-    return st;
+  if (ws_bytes > 0 && (st = stream_workspace(dev, cs, ws_bytes, &ws)) != WF_OK) return st;
+  if (n_split > 1) {
+    uint8_t *base = reinterpret_cast<uint8_t *>(ws) + sched_bytes + vt_bytes;
+    p.part_o = reinterpret_cast<float *>(base);
+    p.part_lse = reinterpret_cast<float *>(base + part_o_bytes);
+    p.part_rows = part_rows;
+  }
   if (dt == WF_F32) {
     float *vt = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(ws) + sched_bytes);
     if (n_keys > 0) {
@@ -434,11 +558,12 @@ wf_status_t wf_attn_fwd_debug(const wf_tensor_t *q, const wf_tensor_t *qRope, co
     p.lq = (int32_t)d.lq;
     p.lk = (int32_t)d.lk;
     const int64_t per_bh = (d.lq + kern.unit_rows - 1) / kern.unit_rows;
-    const int64_t units = per_bh * d.batch * headNum;
-    if (units > INT32_MAX) return fail(WF_ERR_UNSUPPORTED, "too many work units (%lld)", (long long)units);
+    const int64_t units = dense_units;
+    if (units * n_split > INT32_MAX)
+      return fail(WF_ERR_UNSUPPORTED, "too many work items (%lld)", (long long)(units * n_split));
     p.units_per_bh = (int32_t)per_bh;
     p.n_units_dense = (int32_t)units;
-    if (units < grid) grid = (int)units;
+    if (units * n_split < grid) grid = (int)(units * n_split);
   } else {
     const int64_t B = d.batch;
     cudaError_t e = launch_sched_prep(static_cast<const int32_t *>(qSeqLen->data),
@@ -451,6 +576,35 @@ wf_status_t wf_attn_fwd_debug(const wf_tensor_t *q, const wf_tensor_t *qRope, co
   }
   cudaError_t e = kern.launch(p, grid, cs);
   if (e != cudaSuccess) return cuda_fail(e, "attention kernel launch");
+  if (n_split > 1) {
+    MergeParams mp{};
+    mp.parts = p.part_o;
+    mp.p_ss = part_rows * d.dv;
+    mp.p_sr = d.dv;
+    mp.lses = p.part_lse;
+    mp.l_ss = part_rows;
+    mp.l_sr = 1;
+    mp.n_split = n_split;
+    mp.dv = (int32_t)d.dv;
+    mp.rows = part_rows;
+    mp.out = out->data;
+    mp.out_bf16 = dt == WF_BF16;
+    mp.lse = p.lse;
+    if (!d.varlen) {       // row = (b * H + h) * Lq + i
+      mp.n1 = headNum;
+      mp.n2 = d.lq;
+      mp.o_s0 = p.o_sb; mp.o_s1 = p.o_sh; mp.o_s2 = p.o_si;
+      mp.e_s0 = p.l_sb; mp.e_s1 = p.l_sh; mp.e_s2 = p.l_si;
+    } else {               // row = token * H + h
+      mp.n1 = d.tq;
+      mp.n2 = headNum;
+      mp.o_s1 = p.o_si; mp.o_s2 = p.o_sh;
+      mp.e_s1 = p.l_si; mp.e_s2 = p.l_sh;
+      mp.sched = ws;
+      mp.sched_tokens = sl.cu_q + (int32_t)d.batch;
+    }
+    if ((e = launch_merge(mp, cs)) != cudaSuccess) return cuda_fail(e, "merge launch");
+  }
   return WF_OK;
 }
 

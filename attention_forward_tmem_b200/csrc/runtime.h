@@ -19,13 +19,11 @@ wf_status_t cuda_fail(cudaError_t e, const char *what);
 
 size_t dtype_size(int32_t dtype);
 
-// Per-device state: SM count, status word address, schedule workspace.
+// Per-device state: SM count, status word address.
 struct DeviceState {
   int sm_count = 0;
   int cc_major = 0, cc_minor = 0;
   int32_t *status = nullptr;     // address of the device status word
-  int32_t *ws = nullptr;         // schedule workspace
-  size_t ws_bytes = 0;
 };
 // Current device's state (lazily initialised), or nullptr with the error set.
 DeviceState *current_device_state(wf_status_t *st);

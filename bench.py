@@ -17,6 +17,13 @@ workload (independent batches: weak scaling, no collective on the data path);
 
 ``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same
 workload (rank 0 only), the slow baseline arm.
+
+Other workloads (``--workload``): ``mla_varlen_prefill`` (packed MLA, 8
+sequences), ``long_gqa_causal`` (L 65536), and ``blockkv_rolling``: one step
+is the whole 16-chunk rolling-cache loop (cache write + attention of 1024
+queries over up to 8192 visible keys per chunk); it is timed as a CUDA graph
+of that loop, and the line adds the attention-only and cache-write times of a
+step.
 """
 from __future__ import annotations
 
@@ -149,6 +156,23 @@ class ClockSampler:
 
 # ------------------------------------------------------------- workloads
 
+def config_of(name):
+    """The `config` object of the JSON line (both arms)."""
+    w = W.WORKLOADS[name]
+    if name == "mla_varlen_prefill":
+        lens = W.seqlens(w.batch, 512, 4096, W.SEED).tolist()
+        return {"workload": name, "batch": w.batch, "seqlens": lens, "n_tokens": int(sum(lens)),
+                "head_num": w.head_num, "head_dim": w.dqk, "rope_dim": w.drope, "mask": "causal"}
+    if name == "blockkv_rolling":
+        c = W.BLOCKKV
+        return {"workload": name, "batch": 1, "head_num": w.head_num, "head_dim": w.dqk,
+                "chunk_size": c["chunk_size"], "sink_size": c["sink_size"],
+                "window_size": c["window_size"], "n_chunks": c["n_chunks"], "mask": "none",
+                "step": "16 chunks: cache write + attention over the visible keys"}
+    return {"workload": name, "batch": w.batch, "head_num": w.head_num,
+            "kv_head_num": w.kv_head_num, "seq_len": w.seq, "head_dim": w.dqk, "mask": w.mask}
+
+
 class Workload:
     """One step's inputs and the call that runs it through the public API."""
 
@@ -165,9 +189,6 @@ class Workload:
                                      w.dtype, W.SEED, w.input_scale)
             self.host = {"q": q, "k": k, "v": v}
             self.flops = w.batch * w.head_num * 2 * (w.dqk + w.dv) * kept_pairs_causal(w.seq, w.seq)
-            self.config = {"workload": name, "batch": w.batch, "head_num": w.head_num,
-                           "kv_head_num": w.kv_head_num, "seq_len": w.seq, "head_dim": w.dqk,
-                           "mask": "causal"}
         elif name == "mla_varlen_prefill":
             d = W.mla_varlen_prefill()
             self.host = d
@@ -175,11 +196,9 @@ class Workload:
             self.flops = sum(w.head_num * 2 * (w.dqk + w.drope + w.dv) * kept_pairs_causal(L, L)
                              for L in lens)
             self.launches_per_step = 2          # schedule + attention
-            self.config = {"workload": name, "batch": w.batch, "seqlens": lens,
-                           "n_tokens": int(sum(lens)), "head_num": w.head_num,
-                           "head_dim": w.dqk, "rope_dim": w.drope, "mask": "causal"}
         else:
             raise SystemExit(f"bench workload {name!r} is not a single-call workload")
+        self.config = config_of(name)
         self.out_host = None
 
     def to_device(self):
@@ -202,6 +221,122 @@ class Workload:
 
     def host_bytes(self):
         return sum(t.numel() * t.element_size() for t in self.host.values())
+
+
+class RollingWorkload:
+    """The rolling BlockKVCache loop: one step = 16 chunks, each
+    before_update -> update (cache write) -> cached views -> attention of the
+    chunk's 1024 queries over the visible keys (no mask) -> after_update.
+    The cache (sink 1024 + window 7168 positions) is re-created (host state
+    only) at the start of every step, over the same device buffers."""
+
+    def __init__(self, name, device):
+        from attention_forward_tmem_b200 import api
+        self.api = api
+        self.name = name
+        self.device = device
+        self.w = w = W.WORKLOADS[name]
+        c = W.BLOCKKV
+        self.chunk, self.n_chunks = c["chunk_size"], c["n_chunks"]
+        self.sink, self.window = c["sink_size"], c["window_size"]
+        self.cache_len = self.sink + self.window
+        self.host = {}
+        for i in range(self.n_chunks):
+            q, k, v = W.blockkv_chunk(i, w.head_num, self.chunk, w.dqk, w.dtype)
+            self.host[f"q{i}"], self.host[f"k{i}"], self.host[f"v{i}"] = q, k, v
+        self.vis = [min((i + 1) * self.chunk, self.cache_len) for i in range(self.n_chunks)]
+        self.flops = sum(w.head_num * 2 * (w.dqk + w.dv) * self.chunk * n for n in self.vis)
+        self.cache_bytes = self.n_chunks * 2 * 2 * w.head_num * self.chunk * w.dqk * 2  # k+v, read+write
+        self.config = config_of(name)
+
+    def launches_per_chunk(self, i):
+        """Kernels one chunk launches: k and v copies, attention, and the merge
+        pass when the library splits the keys (dense layout, units < SMs)."""
+        sm = torch.cuda.get_device_properties(self.device).multi_processor_count
+        units = self.w.head_num * ((self.chunk + 255) // 256)
+        n = 1
+        if units < sm:
+            n = max(1, min(sm // units, ((self.vis[i] + 127) // 128) // 4))
+        return 3 + (1 if n > 1 else 0)
+
+    @property
+    def launches_per_step(self):
+        return sum(self.launches_per_chunk(i) for i in range(self.n_chunks))
+
+    def to_device(self):
+        self.dev = {k: v.to(self.device) for k, v in self.host.items()}
+        shape = (1, self.w.head_num, self.cache_len, self.w.dqk)
+        self.kb = torch.zeros(shape, dtype=self.w.dtype, device=self.device)
+        self.vb = torch.zeros(shape, dtype=self.w.dtype, device=self.device)
+        self.out = torch.empty((self.n_chunks, 1, self.w.head_num, self.chunk, self.w.dv),
+                               dtype=self.w.dtype, device=self.device)
+
+    def step(self, dev=None, out=None, events=None):
+        d = dev or self.dev
+        out = self.out if out is None else out
+        api = self.api
+        cache = api.BlockKVCache(self.kb, self.vb, chunk_size=self.chunk, window_size=self.window,
+                                 sink_size=self.sink)
+        for i in range(self.n_chunks):
+            if events is not None:
+                torch.cuda._sleep(2_000_000)       # let the host queue the chunk's work
+                events[i][0].record()
+            cache.before_update(i)
+            cache.update(d[f"k{i}"], d[f"v{i}"])
+            if events is not None:
+                events[i][1].record()
+            api.attn_fwd(d[f"q{i}"], cache.cached_k(), cache.cached_v(), mask_type=api.MaskType.NONE,
+                         qk_scale=self.w.qk_scale, out=out[i])
+            if events is not None:
+                events[i][2].record()
+            cache.after_update(i)
+
+    def host_bytes(self):
+        return sum(t.numel() * t.element_size() for t in self.host.values())
+
+    def phase_times(self):
+        """(cache-write ms, attention ms) of one step, from events around each
+        chunk's two phases (the host is kept ahead of the GPU)."""
+        self.step()                 # this stream's library workspace reaches its size
+        torch.cuda.synchronize()
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(self.n_chunks)]
+        self.step(events=ev)
+        torch.cuda.synchronize()
+        write = sum(e[0].elapsed_time(e[1]) for e in ev)
+        attn = sum(e[1].elapsed_time(e[2]) for e in ev)
+        return write, attn
+
+
+def time_device_graph(wl, steps, warmup):
+    """The step captured once in a CUDA graph (after eager warm-up on the
+    capture stream, so that no allocation happens during capture), then
+    replayed: times the device work of the step without the Python launch
+    overhead of its 64+ small calls."""
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for _ in range(warmup):
+            wl.step()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        wl.step()
+    torch.cuda.synchronize()
+    for _ in range(warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        e0.record(stream)
+        for _ in range(steps):
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    wl.api.device_status()
+    del g
+    return ms, clk.summary()
 
 
 def time_device(wl, steps, warmup, dist_on):
@@ -255,36 +390,100 @@ def time_e2e(wl, steps, warmup):
 
 # -------------------------------------------------------------- CPU oracle
 
+def _oracle_rows_dense(w, rng, seed):
+    """Rows of one GQA group of a dense causal workload, each over its full
+    causal key range."""
+    import oracle
+    g = w.head_num // w.kv_head_num
+    q, k, v = W.dense_inputs(1, g, 1, w.seq, w.seq, w.dqk, w.dv, w.dtype, seed, w.input_scale)
+
+    def make(n):
+        rows = np.stack([np.zeros(n, np.int64), rng.integers(0, g, n), rng.integers(0, w.seq, n)], 1)
+        fl = float(sum(2 * (w.dqk + w.dv) * (int(r) + 1) for r in rows[:, 2]))
+        return fl, lambda: oracle.sdpa_rows(q, k, v, rows, mask_kind="causal", qk_scale=w.qk_scale,
+                                            head_num=g, kv_head_num=1)
+    desc = f"one GQA group, rows uniform in [0, {w.seq}), each over its full causal key range"
+    return make, 2 * (w.dqk + w.dv) * w.seq / 2, desc
+
+
+def _oracle_rows_packed(w, rng, seed):
+    """Rows of the packed MLA workload (its sequence lengths; one head, as every
+    head costs the same per row), token-uniform, each over its causal range."""
+    import oracle
+    lens = W.seqlens(w.batch, 512, 4096, seed)
+    d = W.packed_inputs(lens, lens, 1, 1, w.dqk, w.dv, w.drope, w.dtype, seed)
+    L = lens.numpy().astype(np.int64)
+    p = L / L.sum()
+
+    def make(n):
+        b = rng.choice(len(L), size=n, p=p)
+        i = (rng.random(n) * L[b]).astype(np.int64)
+        rows = np.stack([b, np.zeros(n, np.int64), i], 1)
+        fl = float(np.sum(2 * (w.dqk + w.drope + w.dv) * (i + 1)))
+        return fl, lambda: oracle.sdpa_rows(d["q"], d["k"], d["v"], rows, qrope=d["qrope"],
+                                            krope=d["krope"], q_seqlen=lens, kv_seqlen=lens,
+                                            mask_kind="causal", qk_scale=w.qk_scale)
+    desc = "packed MLA sequences (one head), rows token-uniform, each over its causal key range"
+    return make, 2 * (w.dqk + w.drope + w.dv) * float(np.sum(L * L) / np.sum(L)) / 2, desc
+
+
+def _oracle_rows_rolling(w, rng, seed):
+    """Rows of the rolling-cache loop (head 0; every head costs the same per
+    row): chunk uniform, each row over the keys visible at that chunk (logical
+    order; attention is order-free)."""
+    import oracle
+    from oracle.kvcache_model import BlockKVCacheModel
+    c = W.BLOCKKV
+    chunks = [tuple(t[:, :1] for t in W.blockkv_chunk(i, w.head_num, c["chunk_size"], w.dqk, w.dtype))
+              for i in range(c["n_chunks"])]
+    model = BlockKVCacheModel(c["sink_size"] + c["window_size"], c["chunk_size"], c["window_size"],
+                              c["sink_size"])
+    vis_ids = [model.logical_chunks(i) for i in range(c["n_chunks"])]
+
+    def make(n):
+        ci = rng.integers(0, c["n_chunks"], n)
+        calls, fl = [], 0.0
+        for i in sorted(set(ci.tolist())):
+            m = int(np.sum(ci == i))
+            rows = np.stack([np.zeros(m, np.int64), np.zeros(m, np.int64),
+                             rng.integers(0, c["chunk_size"], m)], 1)
+            kk = torch.cat([chunks[j][1] for j in vis_ids[i]], dim=2)
+            vv = torch.cat([chunks[j][2] for j in vis_ids[i]], dim=2)
+            fl += m * 2 * (w.dqk + w.dv) * kk.shape[2]
+            calls.append((chunks[i][0], kk, vv, rows))
+
+        def run():
+            for q, kk, vv, rows in calls:
+                oracle.sdpa_rows(q, kk, vv, rows, qk_scale=w.qk_scale)
+        return fl, run
+    desc = "rolling-cache rows of head 0, chunk uniform, each over the keys visible at its chunk"
+    mean_vis = np.mean([len(v) * c["chunk_size"] for v in vis_ids])
+    return make, 2 * (w.dqk + w.dv) * mean_vis, desc
+
+
 def oracle_sample(name, budget_s=12.0, seed=7):
     """Time the fp64 oracle on rows of the workload (each over its full key
     range) for about `budget_s` seconds.  Returns (TFLOP/s, threads, note)."""
     import oracle
     w = W.WORKLOADS[name]
     rng = np.random.default_rng(seed)
-    if name == "mla_varlen_prefill":
-        raise SystemExit("cpu baseline is defined for the dense workloads")
-    # one GQA group of one batch entry: q [1, G, L, D], k/v [1, 1, L, D]
-    g = w.head_num // w.kv_head_num
-    q, k, v = W.dense_inputs(1, g, 1, w.seq, w.seq, w.dqk, w.dv, w.dtype, seed, w.input_scale)
+    maker = {"mla_varlen_prefill": _oracle_rows_packed,
+             "blockkv_rolling": _oracle_rows_rolling}.get(name, _oracle_rows_dense)
+    make, per_row, desc = maker(w, rng, seed)
 
-    def run(n_rows):
-        rows = np.stack([np.zeros(n_rows, np.int64), rng.integers(0, g, n_rows),
-                         rng.integers(0, w.seq, n_rows)], 1)
-        fl = float(sum(2 * (w.dqk + w.dv) * (int(r) + 1) for r in rows[:, 2]))
+    def run(n):
+        fl, fn = make(n)
         t0 = time.perf_counter()
-        oracle.sdpa_rows(q, k, v, rows, mask_kind="causal", qk_scale=w.qk_scale,
-                         head_num=g, kv_head_num=1)
+        fn()
         return fl, time.perf_counter() - t0
 
-    per_row = 2 * (w.dqk + w.dv) * w.seq / 2   # average causal row
     n = 64
     for share in (0.02, 0.15):                  # calibrate twice, then the timed sample
         fl, dt = run(n)
         n = int(min(400000, max(64, fl / max(dt, 1e-6) * budget_s * share / per_row)))
     n = int(min(400000, max(64, fl / max(dt, 1e-6) * budget_s / per_row)))
     fl, dt = run(n)
-    note = (f"{n} query rows of {name} (one GQA group, rows uniform in [0, {w.seq}), "
-            f"each over its full causal key range), fp64 oracle, {dt:.1f} s")
+    note = f"{n} query rows of {name} ({desc}), fp64 oracle, {dt:.1f} s"
     return fl / dt / 1e12, oracle.oracle_threads(), note
 
 
@@ -308,7 +507,6 @@ def reference_arm(args, rank, world):
     if rank != 0:
         return
     name = args.workload
-    w = W.WORKLOADS[name]
     per_step = []
     note = threads = None
     for i in range(args.warmup + args.steps):
@@ -320,9 +518,7 @@ def reference_arm(args, rank, world):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": name, "batch": w.batch, "head_num": w.head_num,
-                       "kv_head_num": w.kv_head_num, "seq_len": w.seq, "head_dim": w.dqk,
-                       "mask": w.mask, "parallelism": "host cores"},
+            "config": dict(config_of(name), parallelism="host cores"),
             "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                              "sample": note},
             "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -336,7 +532,8 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="gqa_causal_prefill",
-                    choices=["gqa_causal_prefill", "mla_varlen_prefill", "long_gqa_causal"])
+                    choices=["gqa_causal_prefill", "mla_varlen_prefill", "long_gqa_causal",
+                             "blockkv_rolling"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-step-s", type=float, default=3.0)
@@ -351,10 +548,28 @@ def main():
 
     dist_on, rank, world = dist_setup(args)
     device = torch.device("cuda", torch.cuda.current_device())
-    wl = Workload(args.workload, device)
+    rolling = args.workload == "blockkv_rolling"
+    wl = RollingWorkload(args.workload, device) if rolling else Workload(args.workload, device)
     wl.to_device()
 
-    ms, clocks = time_device(wl, args.steps, args.warmup, dist_on)
+    extra = {}
+    if rolling:
+        if dist_on:
+            torch.distributed.barrier()
+        try:
+            ms, clocks = time_device_graph(wl, args.steps, args.warmup)
+            how = "step = CUDA graph of the 16-chunk loop (the kernels the API launches)"
+        except RuntimeError as e:          # capture refused: time the eager loop instead
+            print(f"graph capture failed ({e}); timing the eager loop", file=sys.stderr)
+            ms, clocks = time_device(wl, args.steps, args.warmup, False)
+            how = "step = eager 16-chunk loop (graph capture failed)"
+        write_ms, attn_ms = wl.phase_times()
+        extra = {"attention_ms_per_step": attn_ms, "cache_write_ms_per_step": write_ms,
+                 "attention_tflops": wl.flops / (attn_ms / 1e3) / 1e12,
+                 "cache_write_gbs": wl.cache_bytes / (write_ms / 1e3) / 1e9,
+                 "timing": how + "; phase times from per-chunk events"}
+    else:
+        ms, clocks = time_device(wl, args.steps, args.warmup, dist_on)
     ms = parallel.max_over_ranks(ms, device)
     per_launch_ms = ms / args.steps
     value = wl.flops * world * args.steps / (ms / 1e3) / 1e12
@@ -365,7 +580,9 @@ def main():
     e2e_val = wl.flops * world * e2e_steps / (e2e_ms / 1e3) / 1e12
 
     peaks, peak_kind = measured_peaks()
-    achieved = wl.flops / (per_launch_ms / 1e3) / 1e12
+    # the attention kernel's own rate: per launch, or (rolling cache) over the
+    # attention phases of a step
+    achieved = wl.flops / ((extra["attention_ms_per_step"] if rolling else per_launch_ms) / 1e3) / 1e12
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
                 "traffic": profiled_traffic(args.workload),
@@ -375,7 +592,7 @@ def main():
                 "algorithmic_flops_per_launch": wl.flops}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload != "mla_varlen_prefill":
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, threads, note = oracle_sample(args.workload)
         cpu = {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": note}
 
@@ -397,6 +614,7 @@ def main():
                         "d2h_bytes_per_step": d2h},
                 "clocks": clocks,
                 "gpu_launches": args.steps * wl.launches_per_step}
+        line.update(extra)
         print(json.dumps(line), flush=True)
     if dist_on:
         torch.distributed.destroy_process_group()

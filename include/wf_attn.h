@@ -138,6 +138,60 @@ wf_status_t wf_attn_fwd(const wf_tensor_t *q, const wf_tensor_t *qRope,
                         int32_t maskType, wf_tensor_t *out, void *stream);
 
 /*
+ * wf_attn_fwd_ex -- wf_attn_fwd with the row log-sum-exp as a second output
+ * and a choice of split-KV.  The LSE is what lets results computed over
+ * disjoint key sets be combined (wf_attn_merge): the pages name such uses --
+ * context-parallel attention ([P1] "选择最窄的入口") and calcType RING ([P2]
+ * parameter table) -- without writing the step out.
+ *
+ *   lse: NULL, or WF_F32 with out's shape minus the last dim -- dense
+ *     [B, headNum, Lq], packed [nTokens, headNum] -- any element strides (so a
+ *     head-major [headNum, nTokens] buffer may be passed transposed), 4-byte
+ *     aligned.  lse = ln sum_j exp(x_j) over the row's visible keys, x_j the
+ *     scaled score plus the additive mask; -inf for a row that sees no key.
+ *   numSplits: 0 = automatic (dense layout only: when the work units cannot
+ *     fill the SMs, the keys of every unit are split into as many contiguous
+ *     ranges as fill them, each of at least 4 tiles of 128 keys); 1 = no
+ *     split; 2..128 = that many ranges (both layouts).  With more than one
+ *     range each one writes an fp32 partial result and its LSE to the
+ *     library's per-stream workspace, and a merge pass (as wf_attn_merge)
+ *     writes out and lse.  Results differ from the unsplit ones only by
+ *     rounding.
+ * Everything else, including errors and ownership, as wf_attn_fwd;
+ * wf_attn_fwd is this call with lse = NULL and numSplits = 0.
+ */
+wf_status_t wf_attn_fwd_ex(const wf_tensor_t *q, const wf_tensor_t *qRope,
+                           const wf_tensor_t *k, const wf_tensor_t *kRope,
+                           const wf_tensor_t *v,
+                           const wf_tensor_t *qSeqLen, const wf_tensor_t *kvSeqLen,
+                           const wf_tensor_t *mask,
+                           int32_t headNum, int32_t kvHeadNum, float qkScale,
+                           int32_t maskType, wf_tensor_t *out, wf_tensor_t *lse,
+                           int32_t numSplits, void *stream);
+
+/*
+ * wf_attn_merge -- combine S attention results of the same query rows, each
+ * computed over a different, disjoint set of keys, into the result over all
+ * of them (the step behind the uses named at wf_attn_fwd_ex; it follows from
+ * the softmax definition):
+ *     lse = ln sum_s exp(lseParts[s]),   out = sum_s exp(lseParts[s] - lse) * outParts[s].
+ * A part whose LSE is -inf has weight 0 (its row is not read); a row whose
+ * parts are all -inf gives 0 and -inf.
+ *
+ *   outParts: [S, R, Dv] WF_F32 or WF_BF16, normalised partial results (as
+ *     wf_attn_fwd_ex writes them), last dim contiguous, 16-byte aligned
+ *     pointer and strides.  Dv a multiple of 4.
+ *   lseParts: [S, R] WF_F32, natural log, any strides.
+ *   out: [R, Dv] WF_F32 or WF_BF16, same layout rules as outParts.
+ *   lse: NULL or [R] WF_F32.
+ * Rows of a [B, H, L, Dv] or [T, H, Dv] result are passed flattened to R.
+ * Returns WF_OK once launched (asynchronous); argument errors launch nothing.
+ * All tensors are the caller's.
+ */
+wf_status_t wf_attn_merge(const wf_tensor_t *outParts, const wf_tensor_t *lseParts,
+                          wf_tensor_t *out, wf_tensor_t *lse, void *stream);
+
+/*
  * wf_attn_fwd_debug -- wf_attn_fwd with test switches for the bounded waits
  * (no counterpart on the pages; a diagnostic aid).
  *   debug_flags bit 0: the kernel's copy engine never loads the first K tile,

@@ -163,6 +163,84 @@ def test_empty_input_is_a_no_op(lib):
     assert _call(lib, q, k, v, o) == L.WF_OK
 
 
+def _call_ex(lib, q, k, v, out, lse, splits, *, ql=None, kl=None, mt=L.WF_MASK_NONE):
+    r = lambda x: ctypes.byref(x) if x is not None else None
+    return lib.wf_attn_fwd_ex(r(q), None, r(k), None, r(v), r(ql), r(kl), None, q.shape[1],
+                              k.shape[1], 0.125, mt, ctypes.byref(out), r(lse), splits, None)
+
+
+@pytest.mark.parametrize("case,expect", [
+    ("ok", None),
+    ("lse_wrong_rank", L.WF_ERR_INVALID_ARG),
+    ("lse_wrong_shape", L.WF_ERR_INVALID_ARG),
+    ("lse_bf16", L.WF_ERR_INVALID_ARG),
+    ("lse_misaligned", L.WF_ERR_INVALID_ARG),
+    ("splits_negative", L.WF_ERR_INVALID_ARG),
+    ("splits_too_many", L.WF_ERR_INVALID_ARG),
+    ("packed_lse_shape", L.WF_ERR_INVALID_ARG),
+])
+def test_attn_fwd_ex_argument_errors(lib, case, expect):
+    q, k, v, o = _dense()
+    lse, splits, kw = _t([2, 8, 100], L.WF_F32), 0, {}
+    if case == "lse_wrong_rank":
+        lse = _t([2, 8, 100, 1], L.WF_F32)
+    elif case == "lse_wrong_shape":
+        lse = _t([2, 8, 101], L.WF_F32)
+    elif case == "lse_bf16":
+        lse = _t([2, 8, 100], L.WF_BF16)
+    elif case == "lse_misaligned":
+        lse = _t([2, 8, 100], L.WF_F32, data=ALIGNED + 2)
+    elif case == "splits_negative":
+        splits = -1
+    elif case == "splits_too_many":
+        splits = 129
+    elif case == "packed_lse_shape":
+        q, k, v, o = _t([300, 8, 128]), _t([300, 2, 128]), _t([300, 2, 128]), _t([300, 8, 128])
+        kw.update(ql=_t([3], L.WF_I32), kl=_t([3], L.WF_I32))
+        lse = _t([8, 300], L.WF_F32)              # head-major must be passed transposed
+    st = _call_ex(lib, q, k, v, o, lse, splits, **kw)
+    if expect is None:
+        assert st in (L.WF_ERR_NO_DEVICE, L.WF_OK)
+    else:
+        assert st == expect
+        assert lib.wf_last_error_message()
+
+
+@pytest.mark.parametrize("case,expect", [
+    ("ok", None),
+    ("lse_parts_shape", L.WF_ERR_INVALID_ARG),
+    ("out_shape", L.WF_ERR_INVALID_ARG),
+    ("lse_shape", L.WF_ERR_INVALID_ARG),
+    ("dv_not_mult4", L.WF_ERR_UNSUPPORTED),
+    ("int_parts", L.WF_ERR_UNSUPPORTED),
+    ("parts_rank", L.WF_ERR_INVALID_ARG),
+    ("parts_unaligned_stride", L.WF_ERR_INVALID_ARG),
+])
+def test_merge_argument_errors(lib, case, expect):
+    S, R, dv = 3, 50, 128
+    parts, lp, out, lse = _t([S, R, dv], L.WF_F32), _t([S, R], L.WF_F32), _t([R, dv]), _t([R], L.WF_F32)
+    if case == "lse_parts_shape":
+        lp = _t([S, R + 1], L.WF_F32)
+    elif case == "out_shape":
+        out = _t([R, dv + 8])
+    elif case == "lse_shape":
+        lse = _t([R - 1], L.WF_F32)
+    elif case == "dv_not_mult4":
+        parts, out = _t([S, R, 10], L.WF_F32, strides=[R * 12, 12, 1]), _t([R, 10], strides=[16, 1])
+    elif case == "int_parts":
+        parts = _t([S, R, dv], L.WF_I32)
+    elif case == "parts_rank":
+        parts = _t([S, 2, R // 2, dv], L.WF_F32)
+    elif case == "parts_unaligned_stride":
+        parts = _t([S, R, dv], L.WF_F32, strides=[R * 130, 130, 1])
+    st = lib.wf_attn_merge(ctypes.byref(parts), ctypes.byref(lp), ctypes.byref(out), ctypes.byref(lse), None)
+    if expect is None:
+        assert st in (L.WF_ERR_NO_DEVICE, L.WF_OK)
+    else:
+        assert st == expect
+        assert lib.wf_last_error_message()
+
+
 # ------------------------------------------------------------------ BlockKVCache
 
 def _cache(lib, L_=8, chunk=2, window=6, sink=2, seq_dim=2):
