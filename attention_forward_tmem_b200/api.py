@@ -81,8 +81,8 @@ def _require_cuda(*ts):
 
 def attn_fwd(q, k, v, *, qrope=None, krope=None, q_seqlen=None, kv_seqlen=None, mask=None,
              mask_type=None, head_num=None, kv_head_num=None, qk_scale=None, out=None,
-             return_lse=False, lse=None, num_splits=None, stream=None, debug_flags=0,
-             timeout_cycles=0):
+             return_lse=False, lse=None, num_splits=None, kv_layout=None, stream=None,
+             debug_flags=0, timeout_cycles=0):
     """out = softmax(q k^T * qk_scale + mask) v, see ``include/wf_attn.h``.
 
     Dense: q [B,Hq,Lq,D], k/v [B,Hkv,Lk,D].  Packed: q [T,Hq,D], k/v [Tk,Hkv,D]
@@ -94,13 +94,31 @@ def attn_fwd(q, k, v, *, qrope=None, krope=None, q_seqlen=None, kv_seqlen=None, 
     last dim) also returns the natural-log LSE of every row: ``(out, lse)``.
     ``num_splits``: None/0 automatic split-KV, 1 none, n > 1 forced
     (``wf_attn_fwd_ex``).
+
+    Packed layout extras ("MLA Prefill" parameter table): q / qrope may be
+    given flattened as [T, Hq * D] (then ``head_num`` is required), and K /
+    kRope / V padded as [batch, max_seq, Hkv, D] or, with
+    ``kv_layout="padded"``, flattened as [batch, max_seq, Hkv * D] (then
+    ``kv_head_num`` is required).  These are views, no copies.
     """
     _require_cuda(q, k, v, qrope, krope, q_seqlen, kv_seqlen, mask, out, lse)
     varlen = q_seqlen is not None
+    if varlen and q.dim() == 2:
+        if head_num is None:
+            raise ValueError("flattened q [T, Hq*D] needs head_num")
+        q = q.view(q.shape[0], head_num, -1)
+        if qrope is not None:
+            qrope = qrope.view(qrope.shape[0], head_num, -1)
+    if varlen and kv_layout == "padded" and k.dim() == 3:
+        if kv_head_num is None:
+            raise ValueError("flattened padded k/v [B, S, Hkv*D] needs kv_head_num")
+        k, v = (t.view(t.shape[0], t.shape[1], kv_head_num, -1) for t in (k, v))
+        if krope is not None:
+            krope = krope.view(krope.shape[0], krope.shape[1], kv_head_num, -1)
     if head_num is None:
         head_num = q.shape[1]
     if kv_head_num is None:
-        kv_head_num = k.shape[1]
+        kv_head_num = k.shape[2] if (varlen and k.dim() == 4) else k.shape[1]
     if mask_type is None:
         if mask is None:
             mask_type = MaskType.NONE

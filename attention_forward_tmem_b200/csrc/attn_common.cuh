@@ -27,7 +27,8 @@ constexpr float kRescaleThreshold = 8.0f;   // log2 units
 
 
 struct TileInfo {
-  int32_t b, h, hk, q0, lq, lk, qrow, krow, n_kv, off, tma_b;
+  int32_t b, h, hk, q0, lq, lk, qrow, krow, n_kv, off;
+  int32_t tma_b, kb;   // batch coordinate of the Q / the K and V maps
   int32_t sp, kt0;     // split index, first KV tile of the split (0 without split)
 };
 
@@ -58,6 +59,7 @@ __device__ __forceinline__ TileInfo tile_info(const AttnParams &p, int32_t t, in
     ti.lk = p.lk;
     ti.krow = 0;
     ti.tma_b = ti.b;
+    ti.kb = ti.b;
   } else {
     const int32_t *cu_work = p.ws + p.sl.cu_work;
     int32_t lo = 0, hi = p.batch - 1;                   // last k with cu_work[k] <= t
@@ -70,8 +72,9 @@ __device__ __forceinline__ TileInfo tile_info(const AttnParams &p, int32_t t, in
     const int32_t cq = __ldg(p.ws + p.sl.cu_q + ti.b), ck = __ldg(p.ws + p.sl.cu_k + ti.b);
     ti.lq = __ldg(p.ws + p.sl.cu_q + ti.b + 1) - cq;
     ti.lk = __ldg(p.ws + p.sl.cu_k + ti.b + 1) - ck;
-    ti.krow = ck;
+    ti.krow = p.kv_padded ? 0 : ck;      // padded: sequence b's keys start row 0 of batch b
     ti.tma_b = 0;
+    ti.kb = p.kv_padded ? ti.b : 0;
     n_units = (ti.lq + p.unit_rows - 1) / p.unit_rows;
     ti.hk = r / (n_units * G);
     r -= ti.hk * n_units * G;
@@ -197,7 +200,9 @@ __device__ __forceinline__ float softmax_row(const AttnParams &p, const TileInfo
           const int64_t idx = mrow + (int64_t)(k0 + c) * p.m_sj;
           add = p.mask_dtype == kMaskF32
                     ? reinterpret_cast<const float *>(p.mask)[idx]
-                    : __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(p.mask)[idx]);
+                    : p.mask_dtype == kMaskBF16
+                          ? __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(p.mask)[idx])
+                          : __half2float(reinterpret_cast<const __half *>(p.mask)[idx]);
         }
         x[c] = in ? fmaf(add, kLog2e, __uint_as_float(sr[c]) * p.scale_log2) : -INFINITY;
       }
@@ -261,10 +266,10 @@ __device__ __forceinline__ void store_row(const AttnParams &p, const TileInfo &t
 #pragma unroll
     for (int c = 0; c < DV; c += 8) {
       uint4 v;
-      v.x = pack_bf16x2(o[c + 0] * inv, o[c + 1] * inv);
-      v.y = pack_bf16x2(o[c + 2] * inv, o[c + 3] * inv);
-      v.z = pack_bf16x2(o[c + 4] * inv, o[c + 5] * inv);
-      v.w = pack_bf16x2(o[c + 6] * inv, o[c + 7] * inv);
+      v.x = Elem16<T>::pack2(o[c + 0] * inv, o[c + 1] * inv);
+      v.y = Elem16<T>::pack2(o[c + 2] * inv, o[c + 3] * inv);
+      v.z = Elem16<T>::pack2(o[c + 4] * inv, o[c + 5] * inv);
+      v.w = Elem16<T>::pack2(o[c + 6] * inv, o[c + 7] * inv);
       *reinterpret_cast<uint4 *>(dst + c) = v;
     }
   } else {
@@ -337,14 +342,15 @@ __device__ __forceinline__ void tmem_scale_row(uint32_t taddr, float alpha) {
   }
 }
 
-// P (128 values) into TMEM over the score columns: bf16 pairs (64 columns),
-// or fp32 bits read by the TF32 MMA (128 columns).
-template <bool kTF32>
+// P (128 values) into TMEM over the score columns: 16-bit pairs of the
+// input type T (64 columns), or for T = float the fp32 bits read by the TF32
+// MMA (128 columns).
+template <typename T>
 __device__ __forceinline__ void tmem_store_p(uint32_t taddr, const float (&x)[128]) {
   uint32_t pk[64];
-  if constexpr (!kTF32) {
+  if constexpr (sizeof(T) == 2) {
 #pragma unroll
-    for (int c = 0; c < 64; ++c) pk[c] = pack_bf16x2(x[2 * c], x[2 * c + 1]);
+    for (int c = 0; c < 64; ++c) pk[c] = Elem16<T>::pack2(x[2 * c], x[2 * c + 1]);
     tmem_st_x64(taddr, pk);
   } else {
 #pragma unroll

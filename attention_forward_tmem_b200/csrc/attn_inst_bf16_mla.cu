@@ -1,7 +1,7 @@
-// Explicit instantiations of the two-tile bf16 attention kernel (bf16, mla).
+// Explicit instantiations of the two-tile attention kernel (bf16, mla).
 // Split across files so the kernels compile in parallel.
 #include "attn_pingpong.cuh"
 
 namespace wf {
-template cudaError_t launch_attn_pp<128, 64, 128>(const AttnParams &, int, cudaStream_t);
+template cudaError_t launch_attn_pp<__nv_bfloat16, 128, 64, 128>(const AttnParams &, int, cudaStream_t);
 }  // namespace wf

@@ -123,11 +123,11 @@ __device__ void producer_role(const AttnParams &p, uint8_t *smem, AttnCtrl *ctl,
 #pragma unroll
         for (int a = 0; a < Cfg::kQAtoms; ++a)
           tma_load_4d(kdst + a * Cfg::kAtomBytes, &p.tm_k, &ctl->k_full[st], a * Cfg::kAtomE, krow,
-                      ti.hk, ti.tma_b);
+                      ti.hk, ti.kb);
 #pragma unroll
         for (int a = 0; a < Cfg::kRAtoms; ++a)
           tma_load_4d(kdst + (Cfg::kQAtoms + a) * Cfg::kAtomBytes, &p.tm_kr, &ctl->k_full[st],
-                      a * Cfg::kAtomE, krow, ti.hk, ti.tma_b);
+                      a * Cfg::kAtomE, krow, ti.hk, ti.kb);
         k_last[st] = static_cast<int32_t>(n);
       }
       if (!(ok = bwait(&ctl->v_empty[st], (n + 1) & 1, &ctl->abort, p))) break;
@@ -137,10 +137,10 @@ __device__ void producer_role(const AttnParams &p, uint8_t *smem, AttnCtrl *ctl,
       for (int a = 0; a < Cfg::kVAtoms; ++a) {
         if constexpr (Cfg::kVKMajor)   // V^T: (keys, DV rows) box at key offset a*kAtomE
           tma_load_4d(vdst + a * Cfg::kAtomBytes, &p.tm_v, &ctl->v_full[st], krow + a * Cfg::kAtomE,
-                      0, ti.hk, ti.tma_b);
+                      0, ti.hk, ti.kb);
         else
           tma_load_4d(vdst + a * Cfg::kAtomBytes, &p.tm_v, &ctl->v_full[st], a * Cfg::kAtomE, krow,
-                      ti.hk, ti.tma_b);
+                      ti.hk, ti.kb);
       }
       v_last[st] = static_cast<int32_t>(n);
     }
@@ -265,7 +265,7 @@ __device__ void softmax_role(const AttnParams &p, AttnCtrl *ctl, uint32_t tmem) 
       tmem_ld_x128(tmem + lane_base + sb * 128, sr);
       float x[128];
       const float alpha = softmax_row<0>(p, ti, row, (ti.kt0 + j) * kBlockN, sr, x, m, l);
-      tmem_store_p<Cfg::kTF32>(tmem + lane_base + sb * 128, x);
+      tmem_store_p<T>(tmem + lane_base + sb * 128, x);
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
         // O holds the sum up to tile j-1 once PV[gg-1] is done.
         if (!(ok = bwait(&ctl->pv_done[(gg - 1) & 1], ((gg - 1) >> 1) & 1, &ctl->abort, p))) {

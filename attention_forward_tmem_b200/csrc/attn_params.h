@@ -12,7 +12,9 @@ constexpr int kBlockN = 128;     // keys per KV tile
 constexpr int kThreads = 192;    // warps 0-3 softmax, warp 4 TMA, warp 5 MMA
 
 enum MaskKind : int32_t { kMaskNone = 0, kMaskCausal = 1, kMaskKeep = 2, kMaskAdd = 3 };
-enum MaskDtype : int32_t { kMaskU8 = 0, kMaskF32 = 1, kMaskBF16 = 2 };
+enum MaskDtype : int32_t { kMaskU8 = 0, kMaskF32 = 1, kMaskBF16 = 2, kMaskF16 = 3 };
+// Element types of the kernels and the merge pass.
+enum ElemType : int32_t { kElemF32 = 0, kElemBF16 = 1, kElemF16 = 2 };
 
 // Device status codes (same numbers as wf_status_t).
 constexpr int32_t kDevInvalidArg = 1;
@@ -49,6 +51,7 @@ struct alignas(64) AttnParams {
   int32_t batch, hq, hkv, group;
   int32_t lq, lk;                                // dense lengths
   int32_t varlen;
+  int32_t kv_padded;                             // packed q, K/V [batch, max_seq, heads, D]
   int32_t unit_rows;                             // query rows per work unit (128 or 256)
   int32_t n_units_dense, units_per_bh;           // dense: total units, units per (b, h)
   const int32_t *ws;                             // varlen schedule (device)
@@ -79,7 +82,7 @@ struct AttnKernel {
   int32_t unit_rows;     // query rows per work unit of this kernel
 };
 
-// Kernel for (dtype 0 = f32 / 1 = bf16, dqk, drope, dv); launch == nullptr if none.
+// Kernel for (ElemType, dqk, drope, dv); launch == nullptr if none.
 AttnKernel find_attn_kernel(int dtype, int dqk, int drope, int dv);
 
 // V [rows, heads, batch] x d (element strides) -> V^T [batch][heads][d][ld] (fp32).
@@ -91,7 +94,7 @@ cudaError_t launch_transpose_v(const float *v, int64_t s_row, int64_t s_head, in
 // the output decomposes as r = (i0 * n1 + i1) * n2 + i2.
 struct MergeParams {
   const void *parts;         // [n_split][rows][dv], element strides ss / sr
-  int32_t parts_bf16;        // 0: fp32, 1: bf16
+  int32_t parts_type;        // ElemType
   int64_t p_ss, p_sr;
   const float *lses;         // [n_split][rows], element strides
   int64_t l_ss, l_sr;
@@ -101,7 +104,7 @@ struct MergeParams {
   int32_t sched_tokens;      // the length check failed (word 1), and only rows below
                              // sched[sched_tokens] * n2 (the sequences' tokens) are
   void *out;
-  int32_t out_bf16;
+  int32_t out_type;          // ElemType
   int64_t o_s0, o_s1, o_s2;
   float *lse;                // NULL: not wanted
   int64_t e_s0, e_s1, e_s2;
@@ -109,8 +112,11 @@ struct MergeParams {
 
 cudaError_t launch_merge(const MergeParams &mp, cudaStream_t stream);
 
+// k_max_len: padded K/V, the longest kv length that fits (else any value
+// >= n_k_tokens); lengths above it are rejected like sums past the tensors.
 cudaError_t launch_sched_prep(const int32_t *q_len, const int32_t *k_len, int32_t batch,
-                              int64_t n_q_tokens, int64_t n_k_tokens, int32_t head_num,
+                              int64_t n_q_tokens, int64_t n_k_tokens, int64_t k_max_len,
+                              int32_t head_num,
                               int32_t unit_rows, int32_t *ws, const SchedLayout &sl,
                               int32_t *status, cudaStream_t stream);
 

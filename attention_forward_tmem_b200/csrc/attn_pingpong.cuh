@@ -1,5 +1,5 @@
 // attn_pingpong.cuh -- two-tile ("ping-pong") attention forward for sm_100a,
-// bf16 inputs.
+// 16-bit inputs (bf16 or fp16; P is rounded to the input type).
 //
 // Same operation as attn_kernel.cuh ("Core 注意力" section "选择最窄的入口";
 // "MLA Prefill" parameter table).  A CTA owns a 256-row work unit: two
@@ -33,7 +33,7 @@ constexpr uint32_t kPPOtherRegs = 120;       // warpgroup 2: producer, MMA, 2 id
 // launch: 384 threads x 168 registers = 64512 >= 2*128*200 + 128*96 = 63488
 static_assert(2 * 128 * kPPSoftmaxRegs + 128 * kPPOtherRegs <= kPPThreads * 168, "register split");
 
-template <int DQK, int DROPE, int DV>
+template <typename T, int DQK, int DROPE, int DV>
 struct PPCfg {
   static constexpr int kAtomE = 64;                       // bf16 elements per 128-byte row
   static constexpr int kKStep = 16;
@@ -60,8 +60,8 @@ struct PPCfg {
   static constexpr int kSKStepsR = DROPE / kKStep;
   static constexpr int kPVKSteps = kBlockN / kKStep;
   static constexpr int kNPV = kVAtoms * kAtomE;
-  static constexpr uint32_t kIdescS = instr_desc(1, kBlockM, kBlockN, 0);
-  static constexpr uint32_t kIdescPV = instr_desc(1, kBlockM, kNPV, 1);
+  static constexpr uint32_t kIdescS = instr_desc(Elem16<T>::kFmt, kBlockM, kBlockN, 0);
+  static constexpr uint32_t kIdescPV = instr_desc(Elem16<T>::kFmt, kBlockM, kNPV, 1);
   static constexpr uint32_t kTmemCols = 512;
   // FMA-pipe exp2 share (of 16 columns).  Measured on B200 with waits that
   // suspend instead of spinning, a share of 4/16 cost ~4% at head size 128
@@ -109,11 +109,11 @@ __device__ void pp_producer(const AttnParams &p, uint8_t *smem, PPCtrl *ctl, Pro
 #pragma unroll
     for (int a = 0; a < Cfg::kQAtoms; ++a)
       tma_load_4d(dst + a * Cfg::kAtomBytes, &p.tm_k, &ctl->k_full[st], a * Cfg::kAtomE, krow,
-                  ti.hk, ti.tma_b);
+                  ti.hk, ti.kb);
 #pragma unroll
     for (int a = 0; a < Cfg::kRAtoms; ++a)
       tma_load_4d(dst + (Cfg::kQAtoms + a) * Cfg::kAtomBytes, &p.tm_kr, &ctl->k_full[st],
-                  a * Cfg::kAtomE, krow, ti.hk, ti.tma_b);
+                  a * Cfg::kAtomE, krow, ti.hk, ti.kb);
     log.k_last[st] = static_cast<int32_t>(n);
     return true;
   };
@@ -126,7 +126,7 @@ __device__ void pp_producer(const AttnParams &p, uint8_t *smem, PPCtrl *ctl, Pro
 #pragma unroll
     for (int a = 0; a < Cfg::kVAtoms; ++a)
       tma_load_4d(dst + a * Cfg::kAtomBytes, &p.tm_v, &ctl->v_full[st], a * Cfg::kAtomE, krow,
-                  ti.hk, ti.tma_b);
+                  ti.hk, ti.kb);
     log.v_last[st] = static_cast<int32_t>(n);
     return true;
   };
@@ -287,9 +287,8 @@ __device__ void pp_mma(const AttnParams &p, uint8_t *smem, PPCtrl *ctl, uint32_t
 }
 
 // ------------------------------------------------------------------- softmax
-template <int DV, int kEmuPer16>
+template <typename T, int DV, int kEmuPer16>
 __device__ void pp_softmax(const AttnParams &p, PPCtrl *ctl, uint32_t tmem, int s) {
-  using T = __nv_bfloat16;
   const int32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int32_t r = threadIdx.x & 127;                  // row within the tile = TMEM lane
   const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
@@ -315,7 +314,7 @@ __device__ void pp_softmax(const AttnParams &p, PPCtrl *ctl, uint32_t tmem, int 
       tmem_ld_x128(s_addr, sr);
       float x[128];
       const float alpha = softmax_row<kEmuPer16>(p, ti, row, (ti.kt0 + j) * kBlockN, sr, x, m, l);
-      tmem_store_p<false>(s_addr, x);
+      tmem_store_p<T>(s_addr, x);
       // S_s(j) done implies PV_s(j-1) done: O_s may be rescaled right away.
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) tmem_scale_row<DV>(o_addr, alpha);
       tmem_st_wait();
@@ -337,9 +336,9 @@ __device__ void pp_softmax(const AttnParams &p, PPCtrl *ctl, uint32_t tmem, int 
 }
 
 // --------------------------------------------------------------------- kernel
-template <int DQK, int DROPE, int DV>
+template <typename T, int DQK, int DROPE, int DV>
 __global__ void __launch_bounds__(kPPThreads, 1) attn_fwd_pp_kernel(const __grid_constant__ AttnParams p) {
-  using Cfg = PPCfg<DQK, DROPE, DV>;
+  using Cfg = PPCfg<T, DQK, DROPE, DV>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
@@ -377,7 +376,7 @@ __global__ void __launch_bounds__(kPPThreads, 1) attn_fwd_pp_kernel(const __grid
   ProducerLog plog;
   if (warp < 8) {
     regs_increase<kPPSoftmaxRegs>();
-    pp_softmax<DV, Cfg::kEmuPer16>(p, ctl, tmem, warp >> 2);
+    pp_softmax<T, DV, Cfg::kEmuPer16>(p, ctl, tmem, warp >> 2);
   } else {
     regs_decrease<kPPOtherRegs>();
     if (warp == 8 && (threadIdx.x & 31) == 0) pp_producer<Cfg>(p, smem, ctl, plog);
@@ -399,10 +398,10 @@ __global__ void __launch_bounds__(kPPThreads, 1) attn_fwd_pp_kernel(const __grid
   }
 }
 
-template <int DQK, int DROPE, int DV>
+template <typename T, int DQK, int DROPE, int DV>
 cudaError_t launch_attn_pp(const AttnParams &p, int grid, cudaStream_t stream) {
-  using Cfg = PPCfg<DQK, DROPE, DV>;
-  auto kern = attn_fwd_pp_kernel<DQK, DROPE, DV>;
+  using Cfg = PPCfg<T, DQK, DROPE, DV>;
+  auto kern = attn_fwd_pp_kernel<T, DQK, DROPE, DV>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        Cfg::kSmemBytes);
   if (e != cudaSuccess) return e;

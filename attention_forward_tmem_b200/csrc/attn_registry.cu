@@ -1,7 +1,8 @@
 // attn_registry.cu -- maps (dtype, head sizes) to a compiled attention kernel.
-// bf16 runs the two-tile kernel (256-row work units); fp32 runs the
+// bf16 and fp16 run the two-tile kernel (256-row work units); fp32 runs the
 // single-tile TF32 kernel (128-row work units), whose tiles are twice as large.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "attn_params.h"
 
@@ -9,34 +10,38 @@ namespace wf {
 
 template <typename T, int DQK, int DROPE, int DV>
 cudaError_t launch_attn(const AttnParams &p, int grid, cudaStream_t stream);
-template <int DQK, int DROPE, int DV>
+template <typename T, int DQK, int DROPE, int DV>
 cudaError_t launch_attn_pp(const AttnParams &p, int grid, cudaStream_t stream);
 
 AttnKernel find_attn_kernel(int dtype, int dqk, int drope, int dv) {
-#define WF_CASE_PP(TI, Q, R, V) \
-  if (dtype == TI && dqk == Q && drope == R && dv == V) return {&launch_attn_pp<Q, R, V>, 2 * kBlockM};
+#define WF_CASE_PP(T, TI, Q, R, V) \
+  if (dtype == TI && dqk == Q && drope == R && dv == V) return {&launch_attn_pp<T, Q, R, V>, 2 * kBlockM};
+#define WF_CASE_PP16(Q, R, V) \
+  WF_CASE_PP(__nv_bfloat16, kElemBF16, Q, R, V) \
+  WF_CASE_PP(__half, kElemF16, Q, R, V)
 #define WF_CASE_1T(T, TI, Q, R, V) \
   if (dtype == TI && dqk == Q && drope == R && dv == V) return {&launch_attn<T, Q, R, V>, kBlockM};
-  WF_CASE_PP(1, 64, 0, 64)
-  WF_CASE_PP(1, 64, 0, 96)
-  WF_CASE_PP(1, 64, 0, 128)
-  WF_CASE_PP(1, 96, 0, 64)
-  WF_CASE_PP(1, 96, 0, 96)
-  WF_CASE_PP(1, 96, 0, 128)
-  WF_CASE_PP(1, 128, 0, 64)
-  WF_CASE_PP(1, 128, 0, 96)
-  WF_CASE_PP(1, 128, 0, 128)
-  WF_CASE_PP(1, 128, 64, 128)
-  WF_CASE_1T(float, 0, 64, 0, 64)
-  WF_CASE_1T(float, 0, 64, 0, 96)
-  WF_CASE_1T(float, 0, 64, 0, 128)
-  WF_CASE_1T(float, 0, 96, 0, 64)
-  WF_CASE_1T(float, 0, 96, 0, 96)
-  WF_CASE_1T(float, 0, 96, 0, 128)
-  WF_CASE_1T(float, 0, 128, 0, 64)
-  WF_CASE_1T(float, 0, 128, 0, 96)
-  WF_CASE_1T(float, 0, 128, 0, 128)
+  WF_CASE_PP16(64, 0, 64)
+  WF_CASE_PP16(64, 0, 96)
+  WF_CASE_PP16(64, 0, 128)
+  WF_CASE_PP16(96, 0, 64)
+  WF_CASE_PP16(96, 0, 96)
+  WF_CASE_PP16(96, 0, 128)
+  WF_CASE_PP16(128, 0, 64)
+  WF_CASE_PP16(128, 0, 96)
+  WF_CASE_PP16(128, 0, 128)
+  WF_CASE_PP16(128, 64, 128)
+  WF_CASE_1T(float, kElemF32, 64, 0, 64)
+  WF_CASE_1T(float, kElemF32, 64, 0, 96)
+  WF_CASE_1T(float, kElemF32, 64, 0, 128)
+  WF_CASE_1T(float, kElemF32, 96, 0, 64)
+  WF_CASE_1T(float, kElemF32, 96, 0, 96)
+  WF_CASE_1T(float, kElemF32, 96, 0, 128)
+  WF_CASE_1T(float, kElemF32, 128, 0, 64)
+  WF_CASE_1T(float, kElemF32, 128, 0, 96)
+  WF_CASE_1T(float, kElemF32, 128, 0, 128)
 #undef WF_CASE_PP
+#undef WF_CASE_PP16
 #undef WF_CASE_1T
   return {nullptr, 0};
 }

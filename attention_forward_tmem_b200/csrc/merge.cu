@@ -14,6 +14,7 @@
 // a pass); HBM-bound: it reads S partial rows and writes one.
 #include <cstdint>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "attn_params.h"
 #include "sm100_ptx.cuh"
@@ -25,27 +26,38 @@ constexpr int kMergeWarps = 8;
 constexpr float kLog2eM = 1.4426950408889634f;
 constexpr float kLn2M = 0.6931471805599453f;
 
-__device__ __forceinline__ void load4(const void *base, int64_t idx, bool bf16, float (&v)[4]) {
-  if (bf16) {
-    const uint2 u = *reinterpret_cast<const uint2 *>(reinterpret_cast<const __nv_bfloat16 *>(base) + idx);
-    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
-    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
-    v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
-  } else {
+__device__ __forceinline__ void load4(const void *base, int64_t idx, int32_t type, float (&v)[4]) {
+  if (type == kElemF32) {
     const float4 f = *reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(base) + idx);
     v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+    return;
   }
+  const uint2 u = *reinterpret_cast<const uint2 *>(reinterpret_cast<const uint16_t *>(base) + idx);
+  float2 a, b;
+  if (type == kElemBF16) {
+    a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+    b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+  } else {
+    a = __half22float2(*reinterpret_cast<const __half2 *>(&u.x));
+    b = __half22float2(*reinterpret_cast<const __half2 *>(&u.y));
+  }
+  v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
 }
 
-__device__ __forceinline__ void store4(void *base, int64_t idx, bool bf16, const float (&v)[4]) {
-  if (bf16) {
-    uint2 u;
+__device__ __forceinline__ void store4(void *base, int64_t idx, int32_t type, const float (&v)[4]) {
+  if (type == kElemF32) {
+    *reinterpret_cast<float4 *>(reinterpret_cast<float *>(base) + idx) = make_float4(v[0], v[1], v[2], v[3]);
+    return;
+  }
+  uint2 u;
+  if (type == kElemBF16) {
     u.x = pack_bf16x2(v[0], v[1]);
     u.y = pack_bf16x2(v[2], v[3]);
-    *reinterpret_cast<uint2 *>(reinterpret_cast<__nv_bfloat16 *>(base) + idx) = u;
   } else {
-    *reinterpret_cast<float4 *>(reinterpret_cast<float *>(base) + idx) = make_float4(v[0], v[1], v[2], v[3]);
+    u.x = pack_f16x2(v[0], v[1]);
+    u.y = pack_f16x2(v[2], v[3]);
   }
+  *reinterpret_cast<uint2 *>(reinterpret_cast<uint16_t *>(base) + idx) = u;
 }
 
 __global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(const __grid_constant__ MergeParams mp) {
@@ -78,12 +90,12 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(const __grid_co
         if (ls == -INFINITY) continue;                 // weight 0 (its row may be anything)
         const float w = ex2_approx((ls - top) * kLog2eM) * inv;
         float v[4];
-        load4(mp.parts, s * mp.p_ss + r * mp.p_sr + c, mp.parts_bf16 != 0, v);
+        load4(mp.parts, s * mp.p_ss + r * mp.p_sr + c, mp.parts_type, v);
 #pragma unroll
         for (int e = 0; e < 4; ++e) acc[e] = fmaf(w, v[e], acc[e]);
       }
     }
-    store4(mp.out, obase + c, mp.out_bf16 != 0, acc);
+    store4(mp.out, obase + c, mp.out_type, acc);
   }
   if (mp.lse && lane == 0)
     mp.lse[i0 * mp.e_s0 + i1 * mp.e_s1 + i2 * mp.e_s2] = empty ? -INFINITY : top + __log2f(total) * kLn2M;

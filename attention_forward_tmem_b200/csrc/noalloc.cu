@@ -171,7 +171,7 @@ extern "C" wf_status_t wf_attn_fwd_varlen_noalloc(
   p.sl = sl;
   cudaError_t e = launch_sched_prep(static_cast<const int32_t *>(qSeqLen->data),
                                     static_cast<const int32_t *>(kvSeqLen->data), (int32_t)B, tq,
-                                    tk, headNum, kern.unit_rows, ws, sl, ds->status, cs);
+                                    tk, tk, headNum, kern.unit_rows, ws, sl, ds->status, cs);
   if (e != cudaSuccess) return cuda_fail(e, "sched_prep launch");
   e = kern.launch(p, ds->sm_count, cs);
   if (e != cudaSuccess) return cuda_fail(e, "attention kernel launch");

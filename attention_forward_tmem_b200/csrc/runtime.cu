@@ -140,8 +140,9 @@ wf_status_t make_map(CUtensorMap *map, const void *base, int32_t dtype, int64_t 
                                  (cuuint64_t)(s_batch * es)};
   const cuuint32_t box[4] = {(cuuint32_t)(128 / es), (cuuint32_t)kBlockM, 1, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
-  const CUtensorMapDataType dt =
-      dtype == WF_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const CUtensorMapDataType dt = dtype == WF_F32    ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                 : dtype == WF_F16  ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                    : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   CUresult r = fn(map, dt, 4, const_cast<void *>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -191,8 +192,12 @@ wf_status_t check_tensor(const wf_tensor_t *t, const char *name, int ndim, int32
 constexpr int32_t kMaxSplits = 128;        // largest numSplits accepted
 constexpr int64_t kMinTilesPerSplit = 4;   // automatic split: KV tiles per split, at least
 
+static int32_t elem_type(int32_t dtype) {
+  return dtype == WF_F32 ? kElemF32 : dtype == WF_F16 ? kElemF16 : kElemBF16;
+}
+
 struct Dims {
-  bool varlen;
+  bool varlen, kv_padded;
   int64_t batch, lq, lk, tq, tk, dqk, dv, drope;
 };
 
@@ -244,8 +249,9 @@ wf_status_t wf_attn_merge(const wf_tensor_t *outParts, const wf_tensor_t *lsePar
   wf_status_t st;
   if (!outParts || !lseParts || !out) return fail(WF_ERR_INVALID_ARG, "outParts, lseParts and out are required");
   const int32_t pdt = outParts->dtype, odt = out->dtype;
-  if ((pdt != WF_F32 && pdt != WF_BF16) || (odt != WF_F32 && odt != WF_BF16))
-    return fail(WF_ERR_UNSUPPORTED, "outParts / out dtype must be WF_F32 or WF_BF16");
+  auto float_type = [](int32_t t) { return t == WF_F32 || t == WF_BF16 || t == WF_F16; };
+  if (!float_type(pdt) || !float_type(odt))
+    return fail(WF_ERR_UNSUPPORTED, "outParts / out dtype must be WF_F32, WF_BF16 or WF_F16");
   if ((st = check_tensor(outParts, "outParts", 3, pdt, true)) != WF_OK) return st;
   if ((st = check_tensor(lseParts, "lseParts", 2, WF_F32, false)) != WF_OK) return st;
   if ((st = check_tensor(out, "out", 2, odt, true)) != WF_OK) return st;
@@ -266,7 +272,7 @@ wf_status_t wf_attn_merge(const wf_tensor_t *outParts, const wf_tensor_t *lsePar
   if (!ds) return st;
   MergeParams mp{};
   mp.parts = outParts->data;
-  mp.parts_bf16 = pdt == WF_BF16;
+  mp.parts_type = elem_type(pdt);
   mp.p_ss = outParts->stride[0];
   mp.p_sr = outParts->stride[1];
   mp.lses = static_cast<const float *>(lseParts->data);
@@ -278,7 +284,7 @@ wf_status_t wf_attn_merge(const wf_tensor_t *outParts, const wf_tensor_t *lsePar
   mp.n1 = 1;
   mp.n2 = R;
   mp.out = out->data;
-  mp.out_bf16 = odt == WF_BF16;
+  mp.out_type = elem_type(odt);
   mp.o_s2 = out->stride[0];
   if (lse) {
     mp.lse = static_cast<float *>(lse->data);
@@ -301,8 +307,8 @@ static wf_status_t attn_fwd_impl(const wf_tensor_t *q, const wf_tensor_t *qRope,
   wf_status_t st;
   if (!q || !k || !v || !out) return fail(WF_ERR_INVALID_ARG, "q, k, v and out are required");
   const int32_t dt = q->dtype;
-  if (dt != WF_BF16 && dt != WF_F32)
-    return fail(WF_ERR_UNSUPPORTED, "q dtype %d: only WF_BF16 and WF_F32 are implemented", dt);
+  if (dt != WF_BF16 && dt != WF_F16 && dt != WF_F32)
+    return fail(WF_ERR_UNSUPPORTED, "q dtype %d: only WF_BF16, WF_F16 and WF_F32 are implemented", dt);
   if (maskType < WF_MASK_NONE || maskType > WF_MASK_ADDITIVE)
     return fail(WF_ERR_INVALID_ARG, "maskType %d out of range", maskType);
   if (!std::isfinite(qkScale)) return fail(WF_ERR_INVALID_ARG, "qkScale is not finite");
@@ -316,28 +322,32 @@ static wf_status_t attn_fwd_impl(const wf_tensor_t *q, const wf_tensor_t *qRope,
 
   Dims d{};
   d.varlen = qSeqLen != nullptr;
+  // Packed queries with 4-d K / V: the padded layout [batch, max_seq, kvHead, D]
+  // ("MLA Prefill" table rows K / V: [batch, max_seq, kv_head * D]).
+  d.kv_padded = d.varlen && k->ndim == 4;
   // The TF32 path reads V^T with the key index as the innermost TMA
   // coordinate; a packed sequence may start at any token, which breaks the
   // 16-byte rule on that coordinate, so fp32 is dense-only.
   if (d.varlen && dt == WF_F32)
     return fail(WF_ERR_UNSUPPORTED, "WF_F32 inputs are supported in the dense layout only");
-  const int nd = d.varlen ? 3 : 4;
+  const int nd = d.varlen ? 3 : 4;                     // q / out dims
+  const int knd = d.varlen && !d.kv_padded ? 3 : 4;    // k / v dims
   if ((st = check_tensor(q, "q", nd, dt, true)) != WF_OK) return st;
-  if ((st = check_tensor(k, "k", nd, dt, true)) != WF_OK) return st;
-  if ((st = check_tensor(v, "v", nd, dt, true)) != WF_OK) return st;
+  if ((st = check_tensor(k, "k", knd, dt, true)) != WF_OK) return st;
+  if ((st = check_tensor(v, "v", knd, dt, true)) != WF_OK) return st;
   if ((st = check_tensor(out, "out", nd, dt, true)) != WF_OK) return st;
-  const int hd = nd - 2;   // head dim index: 1 in both layouts
-  const int rd = d.varlen ? 0 : 2;   // row (sequence) dim index
+  const int rd = d.varlen ? 0 : 2;                     // q / out row dim
+  const int khd = d.kv_padded ? 2 : 1;                 // k / v head dim
+  const int krd = !d.varlen ? 2 : (d.kv_padded ? 1 : 0);   // k / v row dim
   if (q->shape[1] != headNum || out->shape[1] != headNum)
     return fail(WF_ERR_INVALID_ARG, "q/out head dim must equal headNum %d", headNum);
-  if (k->shape[1] != kvHeadNum || v->shape[1] != kvHeadNum)
+  if (k->shape[khd] != kvHeadNum || v->shape[khd] != kvHeadNum)
     return fail(WF_ERR_INVALID_ARG, "k/v head dim must equal kvHeadNum %d", kvHeadNum);
-  (void)hd;
   d.dqk = q->shape[nd - 1];
-  d.dv = v->shape[nd - 1];
-  if (k->shape[nd - 1] != d.dqk) return fail(WF_ERR_INVALID_ARG, "q and k head sizes differ");
+  d.dv = v->shape[knd - 1];
+  if (k->shape[knd - 1] != d.dqk) return fail(WF_ERR_INVALID_ARG, "q and k head sizes differ");
   if (out->shape[nd - 1] != d.dv) return fail(WF_ERR_INVALID_ARG, "out and v head sizes differ");
-  if (k->shape[rd] != v->shape[rd]) return fail(WF_ERR_INVALID_ARG, "k and v lengths differ");
+  if (k->shape[krd] != v->shape[krd]) return fail(WF_ERR_INVALID_ARG, "k and v lengths differ");
   if (out->shape[rd] != q->shape[rd]) return fail(WF_ERR_INVALID_ARG, "out and q lengths differ");
   if (!d.varlen) {
     d.batch = q->shape[0];
@@ -354,18 +364,20 @@ static wf_status_t attn_fwd_impl(const wf_tensor_t *q, const wf_tensor_t *qRope,
       return fail(WF_ERR_INVALID_ARG, "qSeqLen / kvSeqLen must be contiguous");
     d.batch = qSeqLen->shape[0];
     d.tq = q->shape[0];
-    d.tk = k->shape[0];
+    d.tk = k->shape[krd];          // packed: kv tokens; padded: max_seq
+    if (d.kv_padded && (k->shape[0] != d.batch || v->shape[0] != d.batch))
+      return fail(WF_ERR_INVALID_ARG, "padded k/v first dim must equal the batch %lld", (long long)d.batch);
   }
   d.drope = 0;
   if (qRope) {
     if ((st = check_tensor(qRope, "qRope", nd, dt, true)) != WF_OK) return st;
-    if ((st = check_tensor(kRope, "kRope", nd, dt, true)) != WF_OK) return st;
+    if ((st = check_tensor(kRope, "kRope", knd, dt, true)) != WF_OK) return st;
     d.drope = qRope->shape[nd - 1];
-    if (kRope->shape[nd - 1] != d.drope) return fail(WF_ERR_INVALID_ARG, "qRope/kRope sizes differ");
-    for (int i = 0; i < nd - 1; ++i) {
+    if (kRope->shape[knd - 1] != d.drope) return fail(WF_ERR_INVALID_ARG, "qRope/kRope sizes differ");
+    for (int i = 0; i < nd - 1; ++i)
       if (qRope->shape[i] != q->shape[i]) return fail(WF_ERR_INVALID_ARG, "qRope shape does not match q");
+    for (int i = 0; i < knd - 1; ++i)
       if (kRope->shape[i] != k->shape[i]) return fail(WF_ERR_INVALID_ARG, "kRope shape does not match k");
-    }
   }
 
   // lse: out's shape without the head-size dim, fp32, any strides
@@ -396,7 +408,8 @@ static wf_status_t attn_fwd_impl(const wf_tensor_t *q, const wf_tensor_t *qRope,
     } else {
       if (mask->dtype == WF_F32) mask_dtype = kMaskF32;
       else if (mask->dtype == WF_BF16 && dt == WF_BF16) mask_dtype = kMaskBF16;
-      else return fail(WF_ERR_INVALID_ARG, "additive mask dtype must be WF_F32 (or WF_BF16 with bf16 q)");
+      else if (mask->dtype == WF_F16 && dt == WF_F16) mask_dtype = kMaskF16;
+      else return fail(WF_ERR_INVALID_ARG, "additive mask dtype must be WF_F32 or q's dtype");
     }
     const int64_t full[4] = {d.batch, headNum, d.lq, d.lk};
     for (int i = 0; i < 4; ++i) {
@@ -411,9 +424,9 @@ static wf_status_t attn_fwd_impl(const wf_tensor_t *q, const wf_tensor_t *qRope,
   }
 
   // supported head sizes
-  if (d.drope && !(d.drope == 64 && d.dqk == 128 && d.dv == 128 && dt == WF_BF16))
-    return fail(WF_ERR_UNSUPPORTED, "rope part needs bf16, Dqk = Dv = 128 and a 64-wide rope");
-  const AttnKernel kern = find_attn_kernel(dt == WF_BF16 ? 1 : 0, (int)d.dqk, (int)d.drope, (int)d.dv);
+  if (d.drope && !(d.drope == 64 && d.dqk == 128 && d.dv == 128 && dt != WF_F32))
+    return fail(WF_ERR_UNSUPPORTED, "rope part needs 16-bit inputs, Dqk = Dv = 128 and a 64-wide rope");
+  const AttnKernel kern = find_attn_kernel(elem_type(dt), (int)d.dqk, (int)d.drope, (int)d.dv);
   if (!kern.launch)
     return fail(WF_ERR_UNSUPPORTED, "head sizes Dqk=%lld Dv=%lld (rope %lld) are not implemented",
                 (long long)d.dqk, (long long)d.dv, (long long)d.drope);
@@ -432,23 +445,25 @@ static wf_status_t attn_fwd_impl(const wf_tensor_t *q, const wf_tensor_t *qRope,
   const int64_t n_keys = d.varlen ? d.tk : d.lk;   // rows of k / v
   // q / k / v maps: (D, rows, heads, batch).  Dense: rows = sequence
   // positions, batch = B.  Packed: rows = tokens of all sequences, batch = 1.
+  // Padded K / V: (D, max_seq, heads, batch), like the dense layout.
   struct MapArgs { int64_t rows, batch, s_row, s_head, s_batch; };
-  auto dims_of = [&](const wf_tensor_t *t, int64_t rows) -> MapArgs {
+  auto dims_of = [&](const wf_tensor_t *t, int64_t rows, bool kv) -> MapArgs {
     if (!d.varlen) return {rows, d.batch, t->stride[2], t->stride[1], t->stride[0]};
+    if (kv && d.kv_padded) return {rows, d.batch, t->stride[1], t->stride[2], t->stride[0]};
     return {rows, 1, t->stride[0], t->stride[1], t->stride[0] * rows};
   };
   auto map_of = [&](CUtensorMap *m, const wf_tensor_t *t, int64_t dd, int64_t rows, int64_t heads,
-                    const char *name) {
-    const MapArgs a = dims_of(t, rows);
+                    bool kv, const char *name) {
+    const MapArgs a = dims_of(t, rows, kv);
     return make_map(m, t->data, dt, dd, a.rows, heads, a.batch, a.s_row, a.s_head, a.s_batch, name);
   };
   const int64_t n_q = d.varlen ? d.tq : d.lq;
-  st = map_of(&p.tm_q, q, d.dqk, n_q, headNum, "q");
-  if (st == WF_OK && d.drope) st = map_of(&p.tm_qr, qRope, d.drope, n_q, headNum, "qRope");
+  st = map_of(&p.tm_q, q, d.dqk, n_q, headNum, false, "q");
+  if (st == WF_OK && d.drope) st = map_of(&p.tm_qr, qRope, d.drope, n_q, headNum, false, "qRope");
   if (st == WF_OK && n_keys > 0) {
-    st = map_of(&p.tm_k, k, d.dqk, n_keys, kvHeadNum, "k");
-    if (st == WF_OK && dt == WF_BF16) st = map_of(&p.tm_v, v, d.dv, n_keys, kvHeadNum, "v");
-    if (st == WF_OK && d.drope) st = map_of(&p.tm_kr, kRope, d.drope, n_keys, kvHeadNum, "kRope");
+    st = map_of(&p.tm_k, k, d.dqk, n_keys, kvHeadNum, true, "k");
+    if (st == WF_OK && dt != WF_F32) st = map_of(&p.tm_v, v, d.dv, n_keys, kvHeadNum, true, "v");
+    if (st == WF_OK && d.drope) st = map_of(&p.tm_kr, kRope, d.drope, n_keys, kvHeadNum, true, "kRope");
   }
   if (st != WF_OK) return st;
   // Maps that are never read (no rope part, or no key at all): copies of q's
@@ -485,6 +500,7 @@ static wf_status_t attn_fwd_impl(const wf_tensor_t *q, const wf_tensor_t *qRope,
   p.hkv = kvHeadNum;
   p.group = headNum / kvHeadNum;
   p.varlen = d.varlen ? 1 : 0;
+  p.kv_padded = d.kv_padded ? 1 : 0;
   p.scale_log2 = qkScale * 1.4426950408889634f;
   p.status = ds->status;
   p.timeout_cycles = timeout_cycles > 0 ? timeout_cycles : (2LL << 30);
@@ -568,8 +584,8 @@ static wf_status_t attn_fwd_impl(const wf_tensor_t *q, const wf_tensor_t *qRope,
     const int64_t B = d.batch;
     cudaError_t e = launch_sched_prep(static_cast<const int32_t *>(qSeqLen->data),
                                       static_cast<const int32_t *>(kvSeqLen->data), (int32_t)B,
-                                      d.tq, d.tk, headNum, kern.unit_rows, ws, sl, ds->status,
-                                      cs);
+                                      d.tq, d.kv_padded ? INT64_MAX : d.tk, d.tk, headNum,
+                                      kern.unit_rows, ws, sl, ds->status, cs);
     if (e != cudaSuccess) return cuda_fail(e, "sched_prep launch");
     p.ws = ws;
     p.sl = sl;
@@ -588,7 +604,7 @@ static wf_status_t attn_fwd_impl(const wf_tensor_t *q, const wf_tensor_t *qRope,
     mp.dv = (int32_t)d.dv;
     mp.rows = part_rows;
     mp.out = out->data;
-    mp.out_bf16 = dt == WF_BF16;
+    mp.out_type = elem_type(dt);
     mp.lse = p.lse;
     if (!d.varlen) {       // row = (b * H + h) * Lq + i
       mp.n1 = headNum;

@@ -5,7 +5,8 @@
 // CTA of 1024 threads:
 //   1. prefix sums of the q and kv lengths, and the work units per sequence
 //      (`unit_rows` query rows each);
-//   2. a length check (non-negative, sums within the tensors);
+//   2. a length check (non-negative, sums within the tensors; with padded K/V
+//      every kv length within the padded length);
 //   3. the sequences ordered by unit count, longest first (counting sort), and
 //      the prefix sums of units x headNum in that order.
 // The attention kernel enumerates its work items from these (see attn_params.h).
@@ -50,7 +51,8 @@ __device__ int64_t block_exclusive_scan(int64_t v, int64_t &excl, int64_t *warp_
 
 __global__ void __launch_bounds__(kSchedThreads) sched_prep_kernel(
     const int32_t *__restrict__ q_len, const int32_t *__restrict__ k_len, int32_t batch,
-    int64_t n_q_tokens, int64_t n_k_tokens, int32_t head_num, int32_t *__restrict__ ws,
+    int64_t n_q_tokens, int64_t n_k_tokens, int64_t k_max_len, int32_t head_num,
+    int32_t *__restrict__ ws,
     int32_t unit_rows, SchedLayout sl, int32_t *__restrict__ status) {
   __shared__ int64_t warp_tot[33];
   __shared__ int32_t hist[kHistBins];
@@ -75,7 +77,7 @@ __global__ void __launch_bounds__(kSchedThreads) sched_prep_kernel(
     if (b < batch) {
       lq = q_len[b];
       lk = k_len[b];
-      if (lq < 0 || lk < 0) atomicOr(&bad, 1);
+      if (lq < 0 || lk < 0 || lk > k_max_len) atomicOr(&bad, 1);
       else atomicAdd(&hist[bin_of(units_of(lq))], 1);
     }
     int64_t eq, ek;
@@ -157,12 +159,12 @@ __global__ void __launch_bounds__(kSchedThreads) sched_prep_kernel(
 }  // namespace
 
 cudaError_t launch_sched_prep(const int32_t *q_len, const int32_t *k_len, int32_t batch,
-                              int64_t n_q_tokens, int64_t n_k_tokens, int32_t head_num,
-                              int32_t unit_rows, int32_t *ws, const SchedLayout &sl,
-                              int32_t *status, cudaStream_t stream) {
+                              int64_t n_q_tokens, int64_t n_k_tokens, int64_t k_max_len,
+                              int32_t head_num, int32_t unit_rows, int32_t *ws,
+                              const SchedLayout &sl, int32_t *status, cudaStream_t stream) {
   static_assert(kHistBins == 4 * kSchedThreads, "scan covers 4 bins per thread");
   sched_prep_kernel<<<1, kSchedThreads, 0, stream>>>(q_len, k_len, batch, n_q_tokens, n_k_tokens,
-                                                     head_num, ws, unit_rows, sl, status);
+                                                     k_max_len, head_num, ws, unit_rows, sl, status);
   return cudaGetLastError();
 }
 

@@ -9,6 +9,7 @@
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 namespace wf {
 
@@ -185,7 +186,8 @@ __device__ __forceinline__ void mma_f16_ts_at(uint32_t d_tmem, uint32_t a_tmem, 
 }
 
 // Instruction descriptor for kind::f16 / kind::tf32 with fp32 accumulation.
-// fmt: 1 = bf16, 2 = tf32.  b_mn_major: B stored MN-major (N contiguous).
+// fmt: 0 = f16, 1 = bf16 (kind::f16), 2 = tf32 (kind::tf32); A and B always
+// share it.  b_mn_major: B stored MN-major (N contiguous).
 __host__ __device__ constexpr uint32_t instr_desc(uint32_t fmt, uint32_t M, uint32_t N,
                                                   uint32_t b_mn_major) {
   return (1u << 4)              // D format: f32
@@ -330,5 +332,25 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&v);
 }
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// The 16-bit element types: MMA operand format code and pair packing
+// (round to nearest even).
+template <typename T>
+struct Elem16;
+template <>
+struct Elem16<__nv_bfloat16> {
+  static constexpr uint32_t kFmt = 1;
+  static __device__ __forceinline__ uint32_t pack2(float lo, float hi) { return pack_bf16x2(lo, hi); }
+};
+template <>
+struct Elem16<__half> {
+  static constexpr uint32_t kFmt = 0;
+  static __device__ __forceinline__ uint32_t pack2(float lo, float hi) { return pack_f16x2(lo, hi); }
+};
 
 }  // namespace wf

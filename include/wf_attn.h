@@ -63,7 +63,7 @@ typedef enum wf_status {
 typedef enum wf_dtype {
     WF_F32 = 0,
     WF_BF16 = 1,
-    WF_F16 = 2,   /* reserved: not accepted by wf_attn_fwd yet */
+    WF_F16 = 2,
     WF_U8 = 3,
     WF_I32 = 4
 } wf_dtype_t;
@@ -105,6 +105,17 @@ typedef struct wf_tensor {
  *     device; if they sum past nTokens / nKvTokens (or are negative) the
  *     call computes nothing and the device status becomes
  *     WF_ERR_INVALID_ARG.
+ *   packed q with padded k / v (4-d k, v and kRope), the [P2] table's
+ *   [batch, max_seq, kv_head * D] form viewed as 4 dims:
+ *     k   [batch, max_seq, kvHeadNum, Dqk]   v [batch, max_seq, kvHeadNum, Dv]
+ *     sequence b's keys are rows [0, kvSeqLen[b]) of entry b; q and out stay
+ *     packed.  A kvSeqLen[b] above max_seq is rejected on the device like an
+ *     over-long sum.
+ *   Keys are read in tiles of 128: K / V rows past a sequence's last key up
+ *   to the tile's end (the next sequence's rows, padding, or rows past the
+ *   last sequence) are loaded and get weight exactly 0.  They must hold
+ *   finite values (0 * Inf is NaN in the product); rows past the end of the
+ *   tensor are never read.
  *
  *   qRope / kRope (MLA, [P2] rows QRope/kRope): NULL, or [.., headNum, 64] /
  *     [.., kvHeadNum, 64] in the same layout as q / k.  Scores are then
@@ -115,10 +126,12 @@ typedef struct wf_tensor {
  *     extent).  Must be NULL otherwise.
  *   headNum % kvHeadNum == 0; query head h reads kv head h / (headNum/kvHeadNum).
  *   qkScale multiplies Q*K^T before the mask is added ([P2] row qkScale).
- *   dtypes: q, k, v, qRope, kRope, out all WF_BF16, or all WF_F32 (the F32
- *     path multiplies on TF32 tensor cores; dense layout only, packed F32
- *     returns WF_ERR_UNSUPPORTED).  Dqk, Dv in {64, 96, 128};
- *     with rope: Dqk = 128, Dv = 128, BF16.
+ *   dtypes: q, k, v, qRope, kRope, out all WF_BF16, all WF_F16 (both
+ *     [P2] table types; P is rounded to the same type before P*V), or all
+ *     WF_F32 (the F32 path multiplies on TF32 tensor cores; dense layout only,
+ *     packed F32 returns WF_ERR_UNSUPPORTED).  Dqk, Dv in {64, 96, 128};
+ *     with rope: Dqk = 128, Dv = 128, 16-bit types.
+ *   Additive mask dtype: WF_F32, or q's dtype when that is 16-bit.
  *   Alignment: every data pointer 16-byte aligned; every stride except the
  *     last a multiple of 16 bytes.
  *   A query row that sees no key (causal with Lq > Lk, or an all-false
@@ -178,11 +191,11 @@ wf_status_t wf_attn_fwd_ex(const wf_tensor_t *q, const wf_tensor_t *qRope,
  * A part whose LSE is -inf has weight 0 (its row is not read); a row whose
  * parts are all -inf gives 0 and -inf.
  *
- *   outParts: [S, R, Dv] WF_F32 or WF_BF16, normalised partial results (as
+ *   outParts: [S, R, Dv] WF_F32, WF_BF16 or WF_F16, normalised partial results (as
  *     wf_attn_fwd_ex writes them), last dim contiguous, 16-byte aligned
  *     pointer and strides.  Dv a multiple of 4.
  *   lseParts: [S, R] WF_F32, natural log, any strides.
- *   out: [R, Dv] WF_F32 or WF_BF16, same layout rules as outParts.
+ *   out: [R, Dv] WF_F32, WF_BF16 or WF_F16, same layout rules as outParts.
  *   lse: NULL or [R] WF_F32.
  * Rows of a [B, H, L, Dv] or [T, H, Dv] result are passed flattened to R.
  * Returns WF_OK once launched (asynchronous); argument errors launch nothing.

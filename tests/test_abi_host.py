@@ -76,10 +76,24 @@ def test_valid_call_reaches_device_check(lib):
     q, k, v, o = _dense()
     st = _call(lib, q, k, v, o, mt=L.WF_MASK_CAUSAL)
     assert st in (L.WF_ERR_NO_DEVICE, L.WF_OK)   # WF_OK only where a B200 is present
+    q, k, v, o = _dense(dtype=L.WF_F16)
+    st = _call(lib, q, k, v, o, mt=L.WF_MASK_ADDITIVE, mask=_t([2, 8, 100, 120], L.WF_F16))
+    assert st in (L.WF_ERR_NO_DEVICE, L.WF_OK)
+    # packed q, padded k / v with rope
+    q, o, qr = _t([300, 8, 128]), _t([300, 8, 128]), _t([300, 8, 64])
+    k, v, kr = _t([3, 160, 2, 128]), _t([3, 160, 2, 128]), _t([3, 160, 2, 64])
+    st = _call(lib, q, k, v, o, qr=qr, kr=kr, ql=_t([3], L.WF_I32), kl=_t([3], L.WF_I32), hk=2,
+               mt=L.WF_MASK_CAUSAL)
+    assert st in (L.WF_ERR_NO_DEVICE, L.WF_OK), lib.wf_last_error_message()
 
 
 @pytest.mark.parametrize("case,expect", [
-    ("f16", L.WF_ERR_UNSUPPORTED),
+    ("i32_inputs", L.WF_ERR_UNSUPPORTED),
+    ("mask_f16_with_bf16", L.WF_ERR_INVALID_ARG),
+    ("padded_batch_mismatch", L.WF_ERR_INVALID_ARG),
+    ("padded_head_mismatch", L.WF_ERR_INVALID_ARG),
+    ("padded_f32", L.WF_ERR_UNSUPPORTED),
+    ("padded_rope_mismatch", L.WF_ERR_INVALID_ARG),
     ("heads_not_divisible", L.WF_ERR_INVALID_ARG),
     ("head_count_mismatch", L.WF_ERR_INVALID_ARG),
     ("dtype_mix", L.WF_ERR_INVALID_ARG),
@@ -104,8 +118,19 @@ def test_valid_call_reaches_device_check(lib):
 def test_argument_errors(lib, case, expect):
     q, k, v, o = _dense()
     kw = {}
-    if case == "f16":
-        q, k, v, o = _dense(dtype=L.WF_F16)
+    if case == "i32_inputs":
+        q, k, v, o = _dense(dtype=L.WF_I32)
+    elif case == "mask_f16_with_bf16":
+        kw.update(mt=L.WF_MASK_ADDITIVE, mask=_t([2, 8, 100, 120], L.WF_F16))
+    elif case in ("padded_batch_mismatch", "padded_head_mismatch", "padded_f32", "padded_rope_mismatch"):
+        dt = L.WF_F32 if case == "padded_f32" else L.WF_BF16
+        q, o = _t([300, 8, 128], dt), _t([300, 8, 128], dt)
+        kb = 4 if case == "padded_batch_mismatch" else 3
+        kh = 4 if case == "padded_head_mismatch" else 2
+        k, v = _t([kb, 160, kh, 128], dt), _t([kb, 160, kh, 128], dt)
+        kw.update(ql=_t([3], L.WF_I32), kl=_t([3], L.WF_I32), hk=2)
+        if case == "padded_rope_mismatch":
+            kw.update(qr=_t([300, 8, 64]), kr=_t([3, 150, 2, 64]))
     elif case == "heads_not_divisible":
         q, k, v, o = _dense(Hq=6, Hk=4)
     elif case == "head_count_mismatch":
