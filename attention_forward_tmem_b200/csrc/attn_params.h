@@ -55,6 +55,8 @@ struct alignas(64) AttnParams {
   int32_t unit_rows;                             // query rows per work unit (128 or 256)
   int32_t n_units_dense, units_per_bh;           // dense: total units, units per (b, h)
   const int32_t *ws;                             // varlen schedule (device)
+  int32_t *counters;                             // two-tile kernel: [next item, CTAs done],
+                                                 // zero before a launch, zero after it
   SchedLayout sl;
   // Split-KV: with n_split > 1 every unit's KV tiles are dealt into n_split
   // contiguous ranges, one work item each (item = unit * n_split + split);

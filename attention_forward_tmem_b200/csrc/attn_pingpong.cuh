@@ -75,9 +75,31 @@ struct PPCtrl {
   uint64_t q_full, q_empty, drain;
   uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
   uint64_t k_full[3], k_empty[3], v_full[3], v_empty[3];
+  uint64_t sched_full[2], sched_empty[2];
+  volatile int32_t sched_item[2];
   uint32_t tmem_base;
   volatile int32_t abort;
 };
+
+// Work items are handed out at run time: the producer thread takes the next
+// item index from a global counter (atomicAdd) and publishes it in a two-slot
+// ring; the MMA thread and the 8 softmax warps read it from there.  Items
+// are thus processed in their enumeration order (locality first, longest
+// unit first) by whichever CTA is free, which keeps the K/V tensors in use at
+// one time few and balances the load.  The last CTA to exit resets the
+// counters for the next launch on the stream.
+constexpr uint32_t kSchedConsumers = 1 + 8;     // MMA thread + one lane per softmax warp
+
+// Consumer side: the next item (or a value >= the item count at the end).
+__device__ __forceinline__ bool pp_next_item(const AttnParams &p, PPCtrl *ctl, uint32_t &it,
+                                             int32_t &t, bool arrive) {
+  const uint32_t k = it & 1;
+  if (!bwait(&ctl->sched_full[k], (it >> 1) & 1, &ctl->abort, p)) return false;
+  t = ctl->sched_item[k];
+  if (arrive) mbar_arrive(&ctl->sched_empty[k]);
+  ++it;
+  return true;
+}
 
 // ------------------------------------------------------------------ producer
 template <typename Cfg>
@@ -131,7 +153,14 @@ __device__ void pp_producer(const AttnParams &p, uint8_t *smem, PPCtrl *ctl, Pro
     return true;
   };
 
-  for (int32_t t = blockIdx.x; t < n_units && ok; t += gridDim.x) {
+  for (uint32_t it = 0;; ++it) {
+    // take the next item and publish it to the other roles
+    const uint32_t k = it & 1;
+    if (!(ok = bwait(&ctl->sched_empty[k], ((it >> 1) + 1) & 1, &ctl->abort, p))) break;
+    const int32_t t = atomicAdd(p.counters, 1);
+    ctl->sched_item[k] = t;
+    mbar_arrive(&ctl->sched_full[k]);
+    if (t >= n_units) break;
     const TileInfo t0 = tile_info(p, t, 0), t1 = tile_info(p, t, 1);
     const int32_t n_max = max(t0.n_kv, t1.n_kv);
     if (n_max == 0) continue;
@@ -236,7 +265,9 @@ __device__ void pp_mma(const AttnParams &p, uint8_t *smem, PPCtrl *ctl, uint32_t
     return true;
   };
 
-  for (int32_t t = blockIdx.x; t < n_units && ok; t += gridDim.x) {
+  for (uint32_t it = 0;;) {
+    int32_t t;
+    if (!(ok = pp_next_item(p, ctl, it, t, true)) || t >= n_units) break;
     const int32_t n[2] = {tile_info(p, t, 0).n_kv, tile_info(p, t, 1).n_kv};
     const int32_t n_max = max(n[0], n[1]);
     if (n_max == 0) continue;
@@ -297,7 +328,12 @@ __device__ void pp_softmax(const AttnParams &p, PPCtrl *ctl, uint32_t tmem, int 
   const int32_t n_units = num_units(p);
   uint32_t cs = 0, co = 0;
   bool ok = true;
-  for (int32_t t = blockIdx.x; t < n_units && ok; t += gridDim.x) {
+  for (uint32_t it = 0;;) {
+    int32_t t;
+    ok = pp_next_item(p, ctl, it, t, false);
+    __syncwarp();
+    if (lane == 0 && ok) mbar_arrive(&ctl->sched_empty[(it - 1) & 1]);
+    if (!ok || t >= n_units) break;
     const TileInfo ti = tile_info(p, t, s);
     const int32_t row = ti.q0 + r;
     const bool row_valid = row < ti.lq;
@@ -361,6 +397,10 @@ __global__ void __launch_bounds__(kPPThreads, 1) attn_fwd_pp_kernel(const __grid
       mbar_init(&ctl->v_full[i], 1);
       mbar_init(&ctl->v_empty[i], 1);
     }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&ctl->sched_full[i], 1);
+      mbar_init(&ctl->sched_empty[i], kSchedConsumers);
+    }
     ctl->abort = 0;
     mbar_fence_init();
   }
@@ -395,6 +435,13 @@ __global__ void __launch_bounds__(kPPThreads, 1) attn_fwd_pp_kernel(const __grid
       if (plog.k_last[s] >= 0) drain_wait(&ctl->k_full[s], plog.k_last[s] & 1, p);
     for (int s = 0; s < Cfg::kVStages; ++s)
       if (plog.v_last[s] >= 0) drain_wait(&ctl->v_full[s], plog.v_last[s] & 1, p);
+    // Every fetch of this CTA has returned; the last CTA out resets the
+    // item counter and the exit count for the next launch.
+    __threadfence();
+    if (atomicAdd(p.counters + 1, 1) == static_cast<int32_t>(gridDim.x) - 1) {
+      atomicExch(p.counters, 0);
+      atomicExch(p.counters + 1, 0);
+    }
   }
 }
 

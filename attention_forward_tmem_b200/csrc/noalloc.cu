@@ -27,22 +27,30 @@ namespace {
 constexpr int64_t kScheduleWords = 65536;          // 256 KiB per device
 
 __device__ __align__(256) int32_t g_noalloc_schedule[kScheduleWords];
+// The attention kernel's work-item counters (zero at load; every launch
+// leaves them zero).
+__device__ __align__(16) int32_t g_noalloc_counters[4];
 
-// Device address of g_noalloc_schedule, looked up once per device (in host
-// code the array's name is only a stand-in, not a device address).
+// Device addresses of the two arrays, looked up once per device (in host
+// code an array's name is only a stand-in, not a device address).
 std::mutex g_mu;
 int32_t *g_sched_ptr[64] = {};
+int32_t *g_counter_ptr[64] = {};
 
-wf_status_t schedule_array(int dev, int32_t **out) {
+wf_status_t schedule_array(int dev, int32_t **out, int32_t **counters) {
   if (dev < 0 || dev >= 64) return fail(WF_ERR_NO_DEVICE, "device index %d out of range", dev);
   std::lock_guard<std::mutex> lock(g_mu);
   if (!g_sched_ptr[dev]) {
-    void *p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_schedule);
+    void *p = nullptr, *c = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_schedule);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(schedule array)");
+    if ((e = cudaGetSymbolAddress(&c, g_noalloc_counters)) != cudaSuccess)
+      return cuda_fail(e, "cudaGetSymbolAddress(counters)");
     g_sched_ptr[dev] = static_cast<int32_t *>(p);
+    g_counter_ptr[dev] = static_cast<int32_t *>(c);
   }
   *out = g_sched_ptr[dev];
+  *counters = g_counter_ptr[dev];
   return WF_OK;
 }
 
@@ -127,7 +135,8 @@ extern "C" wf_status_t wf_attn_fwd_varlen_noalloc(
   int dev = 0;
   cudaGetDevice(&dev);
   int32_t *ws = nullptr;
-  if ((st = schedule_array(dev, &ws)) != WF_OK) return st;
+  int32_t *counters = nullptr;
+  if ((st = schedule_array(dev, &ws, &counters)) != WF_OK) return st;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
 
   AttnParams p;
@@ -169,6 +178,7 @@ extern "C" wf_status_t wf_attn_fwd_varlen_noalloc(
   p.timeout_cycles = 2LL << 30;
   p.ws = ws;
   p.sl = sl;
+  p.counters = counters;
   cudaError_t e = launch_sched_prep(static_cast<const int32_t *>(qSeqLen->data),
                                     static_cast<const int32_t *>(kvSeqLen->data), (int32_t)B, tq,
                                     tk, tk, headNum, kern.unit_rows, ws, sl, ds->status, cs);

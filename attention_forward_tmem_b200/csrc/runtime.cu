@@ -88,8 +88,11 @@ DeviceState *current_device_state(wf_status_t *st) {
   return &g_devices.emplace(dev, ds).first->second;
 }
 
-// Workspace of one (device, stream): varlen schedule tables.  Calls on
-// different streams get different workspaces, so they may overlap.
+// Workspace of one (device, stream): a header with the two-tile kernel's
+// work-item counters, then the varlen schedule tables, V^T (fp32) and the
+// split-KV partials.  Calls on different streams get different workspaces,
+// so they may overlap.
+constexpr size_t kWorkspaceHeader = 256;
 static wf_status_t stream_workspace(int dev, cudaStream_t stream, size_t bytes, int32_t **out) {
   std::lock_guard<std::mutex> lock(g_mu);
   auto &slot = g_workspaces[{dev, stream}];
@@ -106,6 +109,11 @@ static wf_status_t stream_workspace(int dev, cudaStream_t stream, size_t bytes, 
     void *p = nullptr;
     cudaError_t e = cudaMalloc(&p, sz);
     if (e != cudaSuccess) return fail(WF_ERR_NO_MEMORY, "cudaMalloc(%zu): %s", sz, cudaGetErrorString(e));
+    // the header (work-item counters) starts at zero; kernels leave it zero
+    if ((e = cudaMemsetAsync(p, 0, kWorkspaceHeader, stream)) != cudaSuccess) {
+      cudaFree(p);
+      return cuda_fail(e, "cudaMemsetAsync(workspace header)");
+    }
     slot.first = static_cast<int32_t *>(p);
     slot.second = sz;
   }
@@ -540,9 +548,11 @@ static wf_status_t attn_fwd_impl(const wf_tensor_t *q, const wf_tensor_t *qRope,
   const int64_t part_rows = n_split > 1 ? (d.varlen ? d.tq : d.batch * d.lq) * headNum : 0;
   const size_t part_o_bytes = ((size_t)n_split * part_rows * d.dv * 4 + 255) & ~size_t(255);
   const size_t part_l_bytes = ((size_t)n_split * part_rows * 4 + 255) & ~size_t(255);
-  const size_t ws_bytes = sched_bytes + vt_bytes + part_o_bytes + part_l_bytes;
-  int32_t *ws = nullptr;
-  if (ws_bytes > 0 && (st = stream_workspace(dev, cs, ws_bytes, &ws)) != WF_OK) return st;
+  const size_t ws_bytes = kWorkspaceHeader + sched_bytes + vt_bytes + part_o_bytes + part_l_bytes;
+  int32_t *ws_base = nullptr;
+  if ((st = stream_workspace(dev, cs, ws_bytes, &ws_base)) != WF_OK) return st;
+  p.counters = ws_base;
+  int32_t *ws = ws_base + kWorkspaceHeader / 4;      // schedule tables
   if (n_split > 1) {
     uint8_t *base = reinterpret_cast<uint8_t *>(ws) + sched_bytes + vt_bytes;
     p.part_o = reinterpret_cast<float *>(base);
