@@ -72,27 +72,52 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(const __grid_co
   const int64_t i2 = r % mp.n2, i01 = r / mp.n2;
   const int64_t i1 = i01 % mp.n1, i0 = i01 / mp.n1;
 
+  // Weights: lane s holds part s's LSE (parts beyond 32 in further rounds);
+  // the warp reduces the max and the sum by shuffles.
   float top = -INFINITY;
-  for (int s = 0; s < mp.n_split; ++s) top = fmaxf(top, mp.lses[s * mp.l_ss + r * mp.l_sr]);
+  for (int s0 = 0; s0 < mp.n_split; s0 += 32) {
+    const int s = s0 + lane;
+    const float ls = s < mp.n_split ? mp.lses[s * mp.l_ss + r * mp.l_sr] : -INFINITY;
+    top = fmaxf(top, ls);
+  }
+#pragma unroll
+  for (int d = 16; d > 0; d >>= 1) top = fmaxf(top, __shfl_xor_sync(0xffffffffu, top, d));
   const bool empty = top == -INFINITY;
   float total = 0.f;
-  if (!empty)
-    for (int s = 0; s < mp.n_split; ++s)
-      total += ex2_approx((mp.lses[s * mp.l_ss + r * mp.l_sr] - top) * kLog2eM);
+  if (!empty) {
+    for (int s0 = 0; s0 < mp.n_split; s0 += 32) {
+      const int s = s0 + lane;
+      const float ls = s < mp.n_split ? mp.lses[s * mp.l_ss + r * mp.l_sr] : -INFINITY;
+      total += ls == -INFINITY ? 0.f : ex2_approx((ls - top) * kLog2eM);
+    }
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) total += __shfl_xor_sync(0xffffffffu, total, d);
+  }
   const float inv = empty ? 0.f : 1.f / total;
 
   const int64_t obase = i0 * mp.o_s0 + i1 * mp.o_s1 + i2 * mp.o_s2;
   for (int c = lane * 4; c < mp.dv; c += 128) {
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     if (!empty) {
-      for (int s = 0; s < mp.n_split; ++s) {
-        const float ls = mp.lses[s * mp.l_ss + r * mp.l_sr];
-        if (ls == -INFINITY) continue;                 // weight 0 (its row may be anything)
-        const float w = ex2_approx((ls - top) * kLog2eM) * inv;
-        float v[4];
-        load4(mp.parts, s * mp.p_ss + r * mp.p_sr + c, mp.parts_type, v);
+      // four parts' rows in flight at a time
+      for (int s = 0; s < mp.n_split; s += 4) {
+        float v[4][4], w[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) acc[e] = fmaf(w, v[e], acc[e]);
+        for (int k = 0; k < 4; ++k) {
+          w[k] = 0.f;
+          if (s + k < mp.n_split) {
+            const float ls = mp.lses[(s + k) * mp.l_ss + r * mp.l_sr];
+            if (ls != -INFINITY) {                       // weight 0: its row may be anything
+              w[k] = ex2_approx((ls - top) * kLog2eM) * inv;
+              load4(mp.parts, (s + k) * mp.p_ss + r * mp.p_sr + c, mp.parts_type, v[k]);
+            }
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          if (w[k] != 0.f)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[e] = fmaf(w[k], v[k][e], acc[e]);
       }
     }
     store4(mp.out, obase + c, mp.out_type, acc);

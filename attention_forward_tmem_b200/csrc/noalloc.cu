@@ -55,6 +55,12 @@ wf_status_t schedule_array(int dev, int32_t **out, int32_t **counters) {
 }
 
 }  // namespace
+
+cudaError_t reset_noalloc_counters() {
+  const int32_t zero[4] = {0, 0, 0, 0};
+  return cudaMemcpyToSymbol(g_noalloc_counters, zero, sizeof(zero));
+}
+
 }  // namespace wf
 
 using namespace wf;

@@ -647,7 +647,23 @@ wf_status_t wf_get_device_status(void *stream) {
   const int32_t zero = 0;
   if ((e = cudaMemcpy(ds->status, &zero, sizeof(zero), cudaMemcpyHostToDevice)) != cudaSuccess)
     return cuda_fail(e, "clearing the device status");
-  if (v == kDevTimeout) return fail(WF_ERR_TIMEOUT, "a bounded device wait ran out");
+  if (v == kDevTimeout) {
+    // Every CTA of an aborted launch still leaves the work-item counters at
+    // zero; reset them anyway (all workspaces on this device and the fixed
+    // arrays) so that a later call starts clean whatever the abort left.
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if ((e = cudaDeviceSynchronize()) != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+    {
+      std::lock_guard<std::mutex> lock(g_mu);
+      for (auto &kv : g_workspaces)
+        if (kv.first.first == dev && kv.second.first &&
+            (e = cudaMemset(kv.second.first, 0, kWorkspaceHeader)) != cudaSuccess)
+          return cuda_fail(e, "resetting the workspace counters");
+    }
+    if ((e = reset_noalloc_counters()) != cudaSuccess) return cuda_fail(e, "resetting the fixed counters");
+    return fail(WF_ERR_TIMEOUT, "a bounded device wait ran out");
+  }
   if (v == kDevInvalidArg) return fail(WF_ERR_INVALID_ARG, "device-side length check failed");
   if (v != 0) return fail(WF_ERR_CUDA, "device status %d", v);
   return WF_OK;

@@ -31,6 +31,9 @@ DeviceState *current_device_state(wf_status_t *st);
 wf_status_t check_tensor(const wf_tensor_t *t, const char *name, int ndim, int32_t dtype,
                          bool need_tma_layout);
 int64_t numel(const wf_tensor_t *t);
+// Zero the allocation-free entry's work-item counters on the current device
+// (noalloc.cu); used after a launch was aborted.
+cudaError_t reset_noalloc_counters();
 // 4-d TMA map (D, rows, heads, batch), (128 bytes of D) x 128 rows box,
 // 128-byte swizzle, zero fill outside the tensor; strides in elements.
 wf_status_t make_map(CUtensorMap *map, const void *base, int32_t dtype, int64_t d, int64_t rows,

@@ -321,7 +321,9 @@ void wf_kvcache_destroy(wf_kvcache_t *cache);
 /* Synchronize `stream`, then read and clear the current device's status
  * word: WF_OK, WF_ERR_TIMEOUT (a bounded wait inside a kernel ran out; the
  * kernel abandoned its work and the affected output is undefined) or
- * WF_ERR_INVALID_ARG (device-side length check failed). */
+ * WF_ERR_INVALID_ARG (device-side length check failed).  On WF_ERR_TIMEOUT
+ * the call also synchronizes the device and resets the library's device-side
+ * work-item counters, so that later calls start clean. */
 wf_status_t wf_get_device_status(void *stream);
 
 /* Description of the last error on the calling host thread ("" if none). */

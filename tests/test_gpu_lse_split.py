@@ -252,3 +252,21 @@ def test_merge_against_oracle_merge(out_dtype):
     assert np.all(got[:, :, 5] == 0) and np.all(np.isneginf(lse.cpu().numpy()[:, :, 5]))
     fin = ~np.isneginf(ref_lse)
     assert np.abs(lse.cpu().numpy()[fin] - ref_lse[fin]).max() <= 1e-5
+
+
+def test_timeout_during_split_launch_then_clean_split_call():
+    """An automatic-split launch (2 units, 16 KV tiles -> 4 splits) that times
+    out; after the status call the next split launches are correct."""
+    q, k, v = W.dense_inputs(1, 2, 2, 256, 2048, 128, 128, torch.bfloat16, 13, 1.0)
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    s = 1 / math.sqrt(128)
+    api.attn_fwd(qd, kd, vd, qk_scale=s, debug_flags=1, timeout_cycles=20_000_000)
+    with pytest.raises(api.WfError) as e:
+        api.device_status()
+    assert e.value.status == 6
+    for _ in range(2):
+        out, lse = api.attn_fwd(qd, kd, vd, qk_scale=s, return_lse=True, num_splits=4)
+        api.device_status()
+        ref, ref_lse = oracle.sdpa(q, k, v, qk_scale=s, with_lse=True)
+        compare(out, ref, torch.bfloat16, "split after timeout")
+        compare_lse(lse, ref_lse, torch.bfloat16, "split after timeout")
