@@ -53,6 +53,7 @@ SIGNATURES = {
     "wf_kvcache_before_update": (_I32, [_P, _I64]),
     "wf_kvcache_update": (_I32, [_P, _T, _T, _P]),
     "wf_kvcache_cached": (_I32, [_P, _T, _T, ctypes.POINTER(_I64)]),
+    "wf_kvcache_update_attend": (_I32, [_P, _T, _T, _T, _I32, _F32, _T, _P]),
     "wf_kvcache_after_update": (_I32, [_P, _I64]),
     "wf_kvcache_get_state": (_I32, [_P, ctypes.POINTER(_I64), ctypes.POINTER(_I64),
                                     ctypes.POINTER(_I64), ctypes.POINTER(_I64),

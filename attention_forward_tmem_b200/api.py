@@ -252,6 +252,24 @@ class BlockKVCache:
         """Visible values, [B, H, vis, D] view of the buffer (physical ring order)."""
         return self._views()[1]
 
+    def update_attend(self, k, v, q, *, qk_scale=None, head_num=None, out=None, stream=None):
+        """The chunk's update, cached views and attention of ``q`` over the
+        visible keys in one call (``wf_kvcache_update_attend``); returns out
+        [B, Hq, Lq, Dv].  Call after ``before_update``, then ``after_update``."""
+        _require_cuda(k, v, q, out)
+        if head_num is None:
+            head_num = q.shape[1]
+        if qk_scale is None:
+            qk_scale = 1.0 / math.sqrt(q.shape[-1])
+        if out is None:
+            out = torch.empty(q.shape[:3] + (self.v_buf.shape[-1],), dtype=q.dtype, device=q.device)
+        kd, vd, qd, od = describe(k), describe(v), describe(q), describe(out)
+        with torch.cuda.device(self.k_buf.device):
+            _check(L.load().wf_kvcache_update_attend(self._h, ctypes.byref(kd), ctypes.byref(vd),
+                                                     ctypes.byref(qd), int(head_num), float(qk_scale),
+                                                     ctypes.byref(od), _stream(stream)))
+        return out
+
     def after_update(self, chunk_idx: int) -> None:
         _check(L.load().wf_kvcache_after_update(self._h, int(chunk_idx)))
 

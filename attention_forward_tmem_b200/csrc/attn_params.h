@@ -43,6 +43,12 @@ struct SchedLayout {
 struct alignas(64) AttnParams {
   CUtensorMap tm_q, tm_k, tm_v, tm_qr, tm_kr;   // 4-d maps (D, rows, heads, batch);
                                                  // fp32: tm_v maps V^T (rows, D, heads, batch)
+  // Fused cache write (two-tile kernel, dense, no mask): key rows
+  // [fuse_lo, fuse_hi) of K / V are read from tm_kc / tm_vc (the new chunk,
+  // row - fuse_lo) instead of tm_k / tm_v, and the CTAs of the first unit of
+  // each kv head store them into tm_k / tm_v.  fuse_hi == 0: no fusion.
+  CUtensorMap tm_kc, tm_vc;
+  int32_t fuse_lo, fuse_hi;
   void *out;
   int64_t o_sb, o_sh, o_si;                      // element strides of out (batch, head, row)
   const void *mask;

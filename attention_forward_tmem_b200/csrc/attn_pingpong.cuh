@@ -111,6 +111,10 @@ __device__ void pp_producer(const AttnParams &p, uint8_t *smem, PPCtrl *ctl, Pro
     tma_prefetch_map(&p.tm_qr);
     tma_prefetch_map(&p.tm_kr);
   }
+  if (p.fuse_hi > 0) {
+    tma_prefetch_map(&p.tm_kc);
+    tma_prefetch_map(&p.tm_vc);
+  }
   const int32_t n_units = num_units(p);
   uint32_t g = 0, u = 0;
   log.q_last = -1;
@@ -126,12 +130,15 @@ __device__ void pp_producer(const AttnParams &p, uint8_t *smem, PPCtrl *ctl, Pro
       return true;
     }
     const int32_t krow = ti.krow + j * kBlockN;
+    // rows of the new chunk (fused cache write) come from the chunk itself
+    const bool fz = krow >= p.fuse_lo && krow < p.fuse_hi;
+    const CUtensorMap *mk = fz ? &p.tm_kc : &p.tm_k;
+    const int32_t ry = fz ? krow - p.fuse_lo : krow;
     uint8_t *dst = smem + Cfg::kKOff + st * Cfg::kKBytes;
     mbar_arrive_expect_tx(&ctl->k_full[st], Cfg::kKBytes);
 #pragma unroll
     for (int a = 0; a < Cfg::kQAtoms; ++a)
-      tma_load_4d(dst + a * Cfg::kAtomBytes, &p.tm_k, &ctl->k_full[st], a * Cfg::kAtomE, krow,
-                  ti.hk, ti.kb);
+      tma_load_4d(dst + a * Cfg::kAtomBytes, mk, &ctl->k_full[st], a * Cfg::kAtomE, ry, ti.hk, ti.kb);
 #pragma unroll
     for (int a = 0; a < Cfg::kRAtoms; ++a)
       tma_load_4d(dst + (Cfg::kQAtoms + a) * Cfg::kAtomBytes, &p.tm_kr, &ctl->k_full[st],
@@ -143,12 +150,14 @@ __device__ void pp_producer(const AttnParams &p, uint8_t *smem, PPCtrl *ctl, Pro
     const uint32_t gg = g + j, st = gg % Cfg::kVStages, n = gg / Cfg::kVStages;
     if (!bwait(&ctl->v_empty[st], (n + 1) & 1, &ctl->abort, p)) return false;
     const int32_t krow = ti.krow + j * kBlockN;
+    const bool fz = krow >= p.fuse_lo && krow < p.fuse_hi;
+    const CUtensorMap *mv = fz ? &p.tm_vc : &p.tm_v;
+    const int32_t ry = fz ? krow - p.fuse_lo : krow;
     uint8_t *dst = smem + Cfg::kVOff + st * Cfg::kVBytes;
     mbar_arrive_expect_tx(&ctl->v_full[st], Cfg::kVBytes);
 #pragma unroll
     for (int a = 0; a < Cfg::kVAtoms; ++a)
-      tma_load_4d(dst + a * Cfg::kAtomBytes, &p.tm_v, &ctl->v_full[st], a * Cfg::kAtomE, krow,
-                  ti.hk, ti.kb);
+      tma_load_4d(dst + a * Cfg::kAtomBytes, mv, &ctl->v_full[st], a * Cfg::kAtomE, ry, ti.hk, ti.kb);
     log.v_last[st] = static_cast<int32_t>(n);
     return true;
   };
@@ -254,6 +263,30 @@ __device__ void pp_mma(const AttnParams &p, uint8_t *smem, PPCtrl *ctl, uint32_t
   auto wait_v = [&](uint32_t gg) {
     return bwait(&ctl->v_full[gg % Cfg::kVStages], (gg / Cfg::kVStages) & 1, &ctl->abort, p);
   };
+  // Fused cache write: the CTAs of the first unit of each kv head store the
+  // new chunk's K / V tiles from shared memory into the cache as soon as they
+  // have landed; each stage is released only after its store has read it.
+  TileInfo ti0;
+  bool writer = false, pending = false;
+  auto store_tile = [&](bool is_k, uint32_t gg, int32_t jj) {
+    const int32_t krow = ti0.krow + jj * kBlockN;
+    if (!writer || krow < p.fuse_lo || krow >= p.fuse_hi) return;
+    fence_proxy_async();
+    const uint8_t *src = is_k ? smem + Cfg::kKOff + (gg % Cfg::kKStages) * Cfg::kKBytes
+                              : smem + Cfg::kVOff + (gg % Cfg::kVStages) * Cfg::kVBytes;
+    const int atoms = is_k ? Cfg::kQAtoms : Cfg::kVAtoms;
+    for (int a = 0; a < atoms; ++a)
+      tma_store_4d(is_k ? &p.tm_k : &p.tm_v, src + a * Cfg::kAtomBytes, a * Cfg::kAtomE, krow, ti0.hk,
+                   ti0.kb);
+    bulk_commit_group();
+    pending = true;
+  };
+  auto stores_read = [&]() {
+    if (pending) {
+      bulk_wait_read();
+      pending = false;
+    }
+  };
   // PV of tile slot s for KV tile (unit-local) jj; returns false on abort.
   auto do_pv = [&](int s, int32_t jj, int32_t n_s, uint32_t gg) -> bool {
     if (jj == 0 && !bwait(&ctl->o_empty[s], (co[s] + 1) & 1, &ctl->abort, p)) return false;
@@ -268,12 +301,15 @@ __device__ void pp_mma(const AttnParams &p, uint8_t *smem, PPCtrl *ctl, uint32_t
   for (uint32_t it = 0;;) {
     int32_t t;
     if (!(ok = pp_next_item(p, ctl, it, t, true)) || t >= n_units) break;
-    const int32_t n[2] = {tile_info(p, t, 0).n_kv, tile_info(p, t, 1).n_kv};
+    ti0 = tile_info(p, t, 0);
+    const int32_t n[2] = {ti0.n_kv, tile_info(p, t, 1).n_kv};
     const int32_t n_max = max(n[0], n[1]);
     if (n_max == 0) continue;
+    writer = p.fuse_hi > 0 && ti0.q0 == 0 && ti0.h % p.group == 0;
     if (!(ok = bwait(&ctl->q_full, u & 1, &ctl->abort, p))) break;
     if (!(ok = wait_k(g))) break;
     tc_fence_after();
+    store_tile(true, g, 0);
 #pragma unroll
     for (int s = 0; s < 2; ++s) {
       if (n[s] > 0) {
@@ -281,11 +317,14 @@ __device__ void pp_mma(const AttnParams &p, uint8_t *smem, PPCtrl *ctl, uint32_t
         tc_commit(&ctl->s_full[s]);
       }
     }
+    stores_read();
     tc_commit(&ctl->k_empty[g % Cfg::kKStages]);
     for (int32_t j = 1; j < n_max && ok; ++j) {
       const uint32_t gk = g + j, gv = g + j - 1;
       if (!(ok = wait_k(gk))) break;
+      store_tile(true, gk, j);
       if (!(ok = wait_v(gv))) break;
+      store_tile(false, gv, j - 1);
 #pragma unroll
       for (int s = 0; s < 2; ++s) {
         if (j - 1 < n[s] && !(ok = do_pv(s, j - 1, n[s], gv))) break;
@@ -295,6 +334,7 @@ __device__ void pp_mma(const AttnParams &p, uint8_t *smem, PPCtrl *ctl, uint32_t
         }
       }
       if (!ok) break;
+      stores_read();
       tc_commit(&ctl->k_empty[gk % Cfg::kKStages]);
       tc_commit(&ctl->v_empty[gv % Cfg::kVStages]);
     }
@@ -303,16 +343,19 @@ __device__ void pp_mma(const AttnParams &p, uint8_t *smem, PPCtrl *ctl, uint32_t
     tc_commit(&ctl->q_empty);
     const uint32_t gl = g + n_max - 1;
     if (!(ok = wait_v(gl))) break;
+    store_tile(false, gl, n_max - 1);
 #pragma unroll
     for (int s = 0; s < 2; ++s)
       if (n_max - 1 < n[s] && !(ok = do_pv(s, n_max - 1, n[s], gl))) break;
     if (!ok) break;
+    stores_read();
     tc_commit(&ctl->v_empty[gl % Cfg::kVStages]);
     for (int s = 0; s < 2; ++s)
       if (n[s] > 0) ++co[s];
     g += n_max;
     ++u;
   }
+  bulk_wait_all();                 // cache stores complete before the CTA ends
   tc_commit(&ctl->drain);
   drain_wait(&ctl->drain, 0, p);
 }

@@ -243,6 +243,44 @@ static void make_view(const wf_tensor_t *buf, int32_t seq_dim, int64_t vis, wf_t
   out->shape[3] = lv.D; out->stride[3] = buf->stride[3];
 }
 
+wf_status_t wf_kvcache_update_attend(wf_kvcache_t *c, const wf_tensor_t *k, const wf_tensor_t *v,
+                                     const wf_tensor_t *q, int32_t headNum, float qkScale,
+                                     wf_tensor_t *out, void *stream) {
+  clear_error();
+  wf_status_t st;
+  if (!c) return fail(WF_ERR_INVALID_ARG, "cache is NULL");
+  if (c->phase != kBefore) return fail(WF_ERR_ORDER, "update_attend without before_update");
+  if ((st = check_like(k, &c->k, c->seq_dim, c->chunk, "k")) != WF_OK) return st;
+  if ((st = check_like(v, &c->v, c->seq_dim, c->chunk, "v")) != WF_OK) return st;
+  const int64_t vis = visible_len(c, c->current);
+  wf_tensor_t kv, vv, kc, vc;
+  make_view(&c->k, c->seq_dim, vis, &kv);
+  make_view(&c->v, c->seq_dim, vis, &vv);
+  make_view(k, c->seq_dim, c->chunk, &kc);      // the chunk in the logical [B, H, C, D] layout
+  make_view(v, c->seq_dim, c->chunk, &vc);
+  const int64_t lo = slot_of(c, c->current) * c->chunk;
+  const int32_t kv_heads = (int32_t)kv.shape[1];
+  bool declined = false;
+  st = attn_fwd_fused(q, &kv, &vv, &kc, &vc, lo, lo + c->chunk, headNum, kv_heads, qkScale, out, stream,
+                      &declined);
+  if (st != WF_OK) return st;                   // argument error: nothing written
+  if (declined) {                               // not fusable: the copies, then the attention
+    const size_t es = dtype_size(c->k.dtype);
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if ((st = copy_positions(k->data, logical(k, c->seq_dim), 0, c->k.data, logical(&c->k, c->seq_dim),
+                             lo, c->chunk, es, cs)) != WF_OK)
+      return st;
+    if ((st = copy_positions(v->data, logical(v, c->seq_dim), 0, c->v.data, logical(&c->v, c->seq_dim),
+                             lo, c->chunk, es, cs)) != WF_OK)
+      return st;
+    if ((st = wf_attn_fwd(q, nullptr, &kv, nullptr, &vv, nullptr, nullptr, nullptr, headNum, kv_heads,
+                          qkScale, WF_MASK_NONE, out, stream)) != WF_OK)
+      return st;
+  }
+  c->phase = kCached;
+  return WF_OK;
+}
+
 wf_status_t wf_kvcache_cached(wf_kvcache_t *c, wf_tensor_t *k_view, wf_tensor_t *v_view, int64_t *visible) {
   clear_error();
   if (!c) return fail(WF_ERR_INVALID_ARG, "cache is NULL");

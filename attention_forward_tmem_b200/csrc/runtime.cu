@@ -197,6 +197,13 @@ wf_status_t check_tensor(const wf_tensor_t *t, const char *name, int ndim, int32
   return WF_OK;
 }
 
+// The new chunk of a fused cache write (see attn_fwd_fused).
+struct FuseArgs {
+  const wf_tensor_t *k_chunk, *v_chunk;
+  int64_t lo, hi;
+  bool *declined;     // set when the call is valid attention but not fusable
+};
+
 constexpr int32_t kMaxSplits = 128;        // largest numSplits accepted
 constexpr int64_t kMinTilesPerSplit = 4;   // automatic split: KV tiles per split, at least
 
@@ -221,7 +228,7 @@ static wf_status_t attn_fwd_impl(const wf_tensor_t *q, const wf_tensor_t *qRope,
                                  const wf_tensor_t *mask, int32_t headNum, int32_t kvHeadNum,
                                  float qkScale, int32_t maskType, wf_tensor_t *out, wf_tensor_t *lse,
                                  int32_t numSplits, void *stream, uint32_t debug_flags,
-                                 int64_t timeout_cycles);
+                                 int64_t timeout_cycles, const FuseArgs *fuse);
 
 wf_status_t wf_attn_fwd(const wf_tensor_t *q, const wf_tensor_t *qRope, const wf_tensor_t *k,
                         const wf_tensor_t *kRope, const wf_tensor_t *v, const wf_tensor_t *qSeqLen,
@@ -229,7 +236,7 @@ wf_status_t wf_attn_fwd(const wf_tensor_t *q, const wf_tensor_t *qRope, const wf
                         int32_t kvHeadNum, float qkScale, int32_t maskType, wf_tensor_t *out,
                         void *stream) {
   return attn_fwd_impl(q, qRope, k, kRope, v, qSeqLen, kvSeqLen, mask, headNum, kvHeadNum, qkScale,
-                       maskType, out, nullptr, 0, stream, 0u, 0);
+                       maskType, out, nullptr, 0, stream, 0u, 0, nullptr);
 }
 
 wf_status_t wf_attn_fwd_ex(const wf_tensor_t *q, const wf_tensor_t *qRope, const wf_tensor_t *k,
@@ -238,7 +245,7 @@ wf_status_t wf_attn_fwd_ex(const wf_tensor_t *q, const wf_tensor_t *qRope, const
                            int32_t kvHeadNum, float qkScale, int32_t maskType, wf_tensor_t *out,
                            wf_tensor_t *lse, int32_t numSplits, void *stream) {
   return attn_fwd_impl(q, qRope, k, kRope, v, qSeqLen, kvSeqLen, mask, headNum, kvHeadNum, qkScale,
-                       maskType, out, lse, numSplits, stream, 0u, 0);
+                       maskType, out, lse, numSplits, stream, 0u, 0, nullptr);
 }
 
 wf_status_t wf_attn_fwd_debug(const wf_tensor_t *q, const wf_tensor_t *qRope, const wf_tensor_t *k,
@@ -248,8 +255,22 @@ wf_status_t wf_attn_fwd_debug(const wf_tensor_t *q, const wf_tensor_t *qRope, co
                               float qkScale, int32_t maskType, wf_tensor_t *out, void *stream,
                               uint32_t debug_flags, int64_t timeout_cycles) {
   return attn_fwd_impl(q, qRope, k, kRope, v, qSeqLen, kvSeqLen, mask, headNum, kvHeadNum, qkScale,
-                       maskType, out, nullptr, 0, stream, debug_flags, timeout_cycles);
+                       maskType, out, nullptr, 0, stream, debug_flags, timeout_cycles, nullptr);
 }
+
+}  // extern "C"
+
+wf_status_t wf::attn_fwd_fused(const wf_tensor_t *q, const wf_tensor_t *k_view, const wf_tensor_t *v_view,
+                               const wf_tensor_t *k_chunk, const wf_tensor_t *v_chunk, int64_t lo,
+                               int64_t hi, int32_t headNum, int32_t kvHeadNum, float qkScale,
+                               wf_tensor_t *out, void *stream, bool *declined) {
+  *declined = false;
+  const FuseArgs f{k_chunk, v_chunk, lo, hi, declined};
+  return attn_fwd_impl(q, nullptr, k_view, nullptr, v_view, nullptr, nullptr, nullptr, headNum,
+                       kvHeadNum, qkScale, WF_MASK_NONE, out, nullptr, 0, stream, 0u, 0, &f);
+}
+
+extern "C" {
 
 wf_status_t wf_attn_merge(const wf_tensor_t *outParts, const wf_tensor_t *lseParts, wf_tensor_t *out,
                           wf_tensor_t *lse, void *stream) {
@@ -310,7 +331,7 @@ static wf_status_t attn_fwd_impl(const wf_tensor_t *q, const wf_tensor_t *qRope,
                                  const wf_tensor_t *mask, int32_t headNum, int32_t kvHeadNum,
                                  float qkScale, int32_t maskType, wf_tensor_t *out, wf_tensor_t *lse,
                                  int32_t numSplits, void *stream, uint32_t debug_flags,
-                                 int64_t timeout_cycles) {
+                                 int64_t timeout_cycles, const FuseArgs *fuse) {
   clear_error();
   wf_status_t st;
   if (!q || !k || !v || !out) return fail(WF_ERR_INVALID_ARG, "q, k, v and out are required");
@@ -439,6 +460,22 @@ static wf_status_t attn_fwd_impl(const wf_tensor_t *q, const wf_tensor_t *qRope,
     return fail(WF_ERR_UNSUPPORTED, "head sizes Dqk=%lld Dv=%lld (rope %lld) are not implemented",
                 (long long)d.dqk, (long long)d.dv, (long long)d.drope);
 
+  if (fuse) {
+    const int64_t n = fuse->hi - fuse->lo;
+    if (d.varlen || maskType != WF_MASK_NONE || d.drope || dt == WF_F32 || fuse->lo < 0 ||
+        fuse->lo % kBlockN || n <= 0 || n % kBlockN || fuse->hi > d.lk) {
+      *fuse->declined = true;       // dense 16-bit, no mask or rope, 128-key boundaries only
+      return WF_OK;
+    }
+    for (const wf_tensor_t *t : {fuse->k_chunk, fuse->v_chunk}) {
+      if ((st = check_tensor(t, "chunk", 4, dt, true)) != WF_OK) return st;
+      if (t->shape[0] != d.batch || t->shape[1] != kvHeadNum || t->shape[2] != n)
+        return fail(WF_ERR_INVALID_ARG, "chunk must be [B, kvHeadNum, %lld, D]", (long long)n);
+    }
+    if (fuse->k_chunk->shape[3] != d.dqk || fuse->v_chunk->shape[3] != d.dv)
+      return fail(WF_ERR_INVALID_ARG, "chunk head sizes differ from k / v");
+  }
+
   // nothing to compute?
   if (d.batch == 0 || numel(q) == 0) return WF_OK;
 
@@ -474,6 +511,14 @@ static wf_status_t attn_fwd_impl(const wf_tensor_t *q, const wf_tensor_t *qRope,
     if (st == WF_OK && d.drope) st = map_of(&p.tm_kr, kRope, d.drope, n_keys, kvHeadNum, true, "kRope");
   }
   if (st != WF_OK) return st;
+  if (st == WF_OK && fuse) {
+    st = map_of(&p.tm_kc, fuse->k_chunk, d.dqk, fuse->hi - fuse->lo, kvHeadNum, true, "k chunk");
+    if (st == WF_OK) st = map_of(&p.tm_vc, fuse->v_chunk, d.dv, fuse->hi - fuse->lo, kvHeadNum, true, "v chunk");
+    p.fuse_lo = (int32_t)fuse->lo;
+    p.fuse_hi = (int32_t)fuse->hi;
+  }
+  if (st != WF_OK) return st;
+  if (!fuse) p.tm_kc = p.tm_vc = p.tm_q;     // never read
   // Maps that are never read (no rope part, or no key at all): copies of q's
   // so that every descriptor passed to the kernel is well formed.
   if (!d.drope) p.tm_qr = p.tm_q;

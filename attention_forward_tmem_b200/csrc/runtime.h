@@ -31,6 +31,17 @@ DeviceState *current_device_state(wf_status_t *st);
 wf_status_t check_tensor(const wf_tensor_t *t, const char *name, int ndim, int32_t dtype,
                          bool need_tma_layout);
 int64_t numel(const wf_tensor_t *t);
+
+// Attention over a cache view whose key rows [lo, hi) are the new chunk
+// k_chunk / v_chunk ([B, Hkv, hi - lo, D], logical layout), which the kernel
+// reads from there and also stores into the view's rows (fused cache write).
+// Needs the dense layout, no mask, no rope, 16-bit types and lo, hi multiples
+// of 128: otherwise, with arguments that are valid for plain attention, it
+// launches nothing, sets *declined and returns WF_OK.
+wf_status_t attn_fwd_fused(const wf_tensor_t *q, const wf_tensor_t *k_view, const wf_tensor_t *v_view,
+                           const wf_tensor_t *k_chunk, const wf_tensor_t *v_chunk, int64_t lo,
+                           int64_t hi, int32_t headNum, int32_t kvHeadNum, float qkScale,
+                           wf_tensor_t *out, void *stream, bool *declined);
 // Zero the allocation-free entry's work-item counters on the current device
 // (noalloc.cu); used after a launch was aborted.
 cudaError_t reset_noalloc_counters();

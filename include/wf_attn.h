@@ -295,6 +295,29 @@ wf_status_t wf_kvcache_update(wf_kvcache_t *cache, const wf_tensor_t *k,
 wf_status_t wf_kvcache_cached(wf_kvcache_t *cache, wf_tensor_t *k_view,
                               wf_tensor_t *v_view, int64_t *visible_len);
 
+/* wf_kvcache_update_attend -- one chunk's update, cached view and attention
+ * in a single kernel ("Core 注意力", section "Block KV cache 的调用顺序": the
+ * chunk's update -> cached_k / cached_v -> attention over the cached keys).
+ * Call after wf_kvcache_before_update, in place of wf_kvcache_update +
+ * wf_kvcache_cached + wf_attn_fwd; follow with wf_kvcache_after_update.
+ *   k, v: the chunk, as for wf_kvcache_update.
+ *   q, out: [B, headNum, Lq, Dqk / Dv] (dense layout of wf_attn_fwd); the
+ *     cache's head count is kvHeadNum.  Attention without a mask over the
+ *     visible keys in physical ring order, as wf_attn_fwd over the
+ *     wf_kvcache_cached views.
+ * The attention kernel reads the chunk's keys and values from k / v directly
+ * and stores them into the ring slot as it goes, so no separate copy runs.
+ * That needs 16-bit buffers and a chunk size that is a multiple of 128;
+ * otherwise the call runs the copy and then wf_attn_fwd (same results).
+ * Results and cache contents are bit-identical to the unfused calls.
+ * WF_ERR_ORDER out of phase; argument errors as wf_kvcache_update /
+ * wf_attn_fwd, with nothing written.  On success the cache is in the state
+ * wf_kvcache_cached leaves it in. */
+wf_status_t wf_kvcache_update_attend(wf_kvcache_t *cache, const wf_tensor_t *k,
+                                     const wf_tensor_t *v, const wf_tensor_t *q,
+                                     int32_t headNum, float qkScale, wf_tensor_t *out,
+                                     void *stream);
+
 /* Commit chunk `chunk_idx` (must equal the one in progress). Host only. */
 wf_status_t wf_kvcache_after_update(wf_kvcache_t *cache, int64_t chunk_idx);
 

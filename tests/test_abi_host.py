@@ -293,6 +293,9 @@ def test_cache_order_errors_on_host(lib):
     assert state() == s0
     kv = _t([1, 2, 2, 4], L.WF_F32)
     assert lib.wf_kvcache_update(h, ctypes.byref(kv), ctypes.byref(kv), None) == L.WF_ERR_ORDER
+    qd = _t([1, 2, 2, 4], L.WF_F32)
+    assert lib.wf_kvcache_update_attend(h, ctypes.byref(kv), ctypes.byref(kv), ctypes.byref(qd), 2, 0.5,
+                                        ctypes.byref(qd), None) == L.WF_ERR_ORDER
     assert lib.wf_kvcache_cached(h, None, None, None) == L.WF_ERR_ORDER
     assert lib.wf_kvcache_after_update(h, 0) == L.WF_ERR_ORDER
     assert state() == s0
