@@ -20,10 +20,11 @@ workload (rank 0 only), the slow baseline arm.
 
 Other workloads (``--workload``): ``mla_varlen_prefill`` (packed MLA, 8
 sequences), ``long_gqa_causal`` (L 65536), and ``blockkv_rolling``: one step
-is the whole 16-chunk rolling-cache loop (cache write + attention of 1024
-queries over up to 8192 visible keys per chunk); it is timed as a CUDA graph
-of that loop, and the line adds the attention-only and cache-write times of a
-step.
+is the whole 16-chunk rolling-cache loop through the fused chunk call (the
+cache write and the attention of 1024 queries over up to 8192 visible keys in
+one kernel per chunk); it is timed as a CUDA graph of that loop, and the line
+adds the same loop through the separate calls (copy kernels, then attention)
+with their phase times.
 """
 from __future__ import annotations
 
@@ -250,14 +251,15 @@ class RollingWorkload:
         self.config = config_of(name)
 
     def launches_per_chunk(self, i):
-        """Kernels one chunk launches: k and v copies, attention, and the merge
-        pass when the library splits the keys (dense layout, units < SMs)."""
+        """Kernels one chunk launches: the attention kernel (which also writes
+        the chunk into the cache), and the merge pass when the library splits
+        the keys (dense layout, units < SMs)."""
         sm = torch.cuda.get_device_properties(self.device).multi_processor_count
         units = self.w.head_num * ((self.chunk + 255) // 256)
         n = 1
         if units < sm:
             n = max(1, min(sm // units, ((self.vis[i] + 127) // 128) // 4))
-        return 3 + (1 if n > 1 else 0)
+        return 1 + (1 if n > 1 else 0)
 
     @property
     def launches_per_step(self):
@@ -271,7 +273,21 @@ class RollingWorkload:
         self.out = torch.empty((self.n_chunks, 1, self.w.head_num, self.chunk, self.w.dv),
                                dtype=self.w.dtype, device=self.device)
 
-    def step(self, dev=None, out=None, events=None):
+    def step(self, dev=None, out=None):
+        """The chunk loop through the fused call (cache write + attention in
+        one kernel per chunk)."""
+        d = dev or self.dev
+        out = self.out if out is None else out
+        cache = self.api.BlockKVCache(self.kb, self.vb, chunk_size=self.chunk, window_size=self.window,
+                                      sink_size=self.sink)
+        for i in range(self.n_chunks):
+            cache.before_update(i)
+            cache.update_attend(d[f"k{i}"], d[f"v{i}"], d[f"q{i}"], qk_scale=self.w.qk_scale, out=out[i])
+            cache.after_update(i)
+
+    def step_unfused(self, dev=None, out=None, events=None):
+        """The same loop as separate calls: update (copy kernels), cached
+        views, attention."""
         d = dev or self.dev
         out = self.out if out is None else out
         api = self.api
@@ -297,30 +313,31 @@ class RollingWorkload:
     def phase_times(self):
         """(cache-write ms, attention ms) of one step, from events around each
         chunk's two phases (the host is kept ahead of the GPU)."""
-        self.step()                 # this stream's library workspace reaches its size
+        self.step_unfused()         # this stream's library workspace reaches its size
         torch.cuda.synchronize()
         ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(self.n_chunks)]
-        self.step(events=ev)
+        self.step_unfused(events=ev)
         torch.cuda.synchronize()
         write = sum(e[0].elapsed_time(e[1]) for e in ev)
         attn = sum(e[1].elapsed_time(e[2]) for e in ev)
         return write, attn
 
 
-def time_device_graph(wl, steps, warmup):
+def time_device_graph(wl, steps, warmup, step=None):
     """The step captured once in a CUDA graph (after eager warm-up on the
     capture stream, so that no allocation happens during capture), then
     replayed: times the device work of the step without the Python launch
-    overhead of its 64+ small calls."""
+    overhead of its many small calls."""
+    step = step or wl.step
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(s):
         for _ in range(warmup):
-            wl.step()
+            step()
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=s):
-        wl.step()
+        step()
     torch.cuda.synchronize()
     for _ in range(warmup):
         g.replay()
@@ -537,6 +554,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-step-s", type=float, default=3.0)
+    ap.add_argument("--no-extras", action="store_true",
+                    help="time the product step only (no e2e, CPU baseline or comparison loop; for profilers)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be at least 3")
@@ -558,31 +577,37 @@ def main():
             torch.distributed.barrier()
         try:
             ms, clocks = time_device_graph(wl, args.steps, args.warmup)
+            ms_unf = None if args.no_extras else time_device_graph(wl, args.steps, args.warmup,
+                                                                   wl.step_unfused)[0]
             how = "step = CUDA graph of the 16-chunk loop (the kernels the API launches)"
         except RuntimeError as e:          # capture refused: time the eager loop instead
             print(f"graph capture failed ({e}); timing the eager loop", file=sys.stderr)
             ms, clocks = time_device(wl, args.steps, args.warmup, False)
+            ms_unf = None
             how = "step = eager 16-chunk loop (graph capture failed)"
-        write_ms, attn_ms = wl.phase_times()
-        extra = {"attention_ms_per_step": attn_ms, "cache_write_ms_per_step": write_ms,
-                 "attention_tflops": wl.flops / (attn_ms / 1e3) / 1e12,
-                 "cache_write_gbs": wl.cache_bytes / (write_ms / 1e3) / 1e9,
-                 "timing": how + "; phase times from per-chunk events"}
+        write_ms, attn_ms = (float("nan"), float("nan")) if args.no_extras else wl.phase_times()
+        extra = {"fused_cache_write": True,
+                 "unfused_ms_per_step": ms_unf / args.steps if ms_unf else None,
+                 "unfused_attention_ms_per_step": attn_ms, "unfused_cache_write_ms_per_step": write_ms,
+                 "unfused_cache_write_gbs": wl.cache_bytes / (write_ms / 1e3) / 1e9,
+                 "timing": how + "; unfused phase times from per-chunk events"}
     else:
         ms, clocks = time_device(wl, args.steps, args.warmup, dist_on)
     ms = parallel.max_over_ranks(ms, device)
     per_launch_ms = ms / args.steps
     value = wl.flops * world * args.steps / (ms / 1e3) / 1e12
 
-    e2e_steps = max(3, min(args.steps, 20))
-    e2e_ms, h2d, d2h = time_e2e(wl, e2e_steps, 3)
-    e2e_ms = parallel.max_over_ranks(e2e_ms, device)
-    e2e_val = wl.flops * world * e2e_steps / (e2e_ms / 1e3) / 1e12
+    e2e_val = h2d = d2h = None
+    if not args.no_extras:
+        e2e_steps = max(3, min(args.steps, 20))
+        e2e_ms, h2d, d2h = time_e2e(wl, e2e_steps, 3)
+        e2e_ms = parallel.max_over_ranks(e2e_ms, device)
+        e2e_val = wl.flops * world * e2e_steps / (e2e_ms / 1e3) / 1e12
 
     peaks, peak_kind = measured_peaks()
-    # the attention kernel's own rate: per launch, or (rolling cache) over the
-    # attention phases of a step
-    achieved = wl.flops / ((extra["attention_ms_per_step"] if rolling else per_launch_ms) / 1e3) / 1e12
+    # the attention kernel's own rate: per launch, or (rolling cache) per step
+    # of fused attention + cache-write kernels and their merge passes
+    achieved = wl.flops / (per_launch_ms / 1e3) / 1e12
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
                 "traffic": profiled_traffic(args.workload),
@@ -592,7 +617,7 @@ def main():
                 "algorithmic_flops_per_launch": wl.flops}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.no_extras:
         v, threads, note = oracle_sample(args.workload)
         cpu = {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": note}
 
