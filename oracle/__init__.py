@@ -11,6 +11,8 @@ Contents:
   * ``brute``                 -- pure-Python per-element loops for tiny inputs
   * ``kvcache_model``         -- plain Python model of the BlockKVCache contract
   * ``merge``                 -- fp64 merge of results over disjoint key sets (by LSE)
+  * ``dca``                   -- fp64 dual chunk attention (three query forms by chunk distance)
 """
 from .sdpa import sdpa, sdpa_rows, build_oracle, oracle_threads, MASK_KINDS  # noqa: F401
 from .merge import merge, MERGE_PLANTS  # noqa: F401
+from .dca import dca, DCA_PLANTS  # noqa: F401

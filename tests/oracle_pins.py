@@ -335,6 +335,51 @@ def pin_merge_closed_forms(plant=0):
 
 MERGE_PINS = [pin_merge_random_key_sets, pin_merge_causal_halves, pin_merge_closed_forms]
 
+
+# --------------------------------------------------------------- DCA pins
+
+def pin_dca_equal_queries_is_causal_attention(plant=0):
+    """All three query forms equal: plain causal attention (torch, GQA)."""
+    g = _rng(60)
+    q, k, v = _randn(g, 1, 4, 21, 8), _randn(g, 1, 2, 21, 8), _randn(g, 1, 2, 21, 5)
+    out = oracle.dca(q, q, q, k, v, chunk=4, qk_scale=0.4, plant=plant)
+    tril = torch.ones(21, 21, dtype=torch.bool).tril()
+    return _close(out, _torch_ref(q, k, v, 0.4, mask=tril).numpy())
+
+
+def pin_dca_one_chunk_is_intra_only(plant=0):
+    """A chunk at least the sequence long: only the intra-chunk form is used."""
+    g = _rng(61)
+    qi, qs, qe = _randn(g, 1, 2, 9, 8), _randn(g, 1, 2, 9, 8), _randn(g, 1, 2, 9, 8)
+    k, v = _randn(g, 1, 2, 9, 8), _randn(g, 1, 2, 9, 6)
+    out = oracle.dca(qi, qs, qe, k, v, chunk=9, qk_scale=0.3, plant=plant)
+    tril = torch.ones(9, 9, dtype=torch.bool).tril()
+    return _close(out, _torch_ref(qi, k, v, 0.3, mask=tril).numpy())
+
+
+def pin_dca_brute_force(plant=0):
+    """Independent per-element loop: the query form picked key by key."""
+    g = _rng(62)
+    qi, qs, qe = _randn(g, 1, 2, 11, 3), _randn(g, 1, 2, 11, 3), _randn(g, 1, 2, 11, 3)
+    k, v = _randn(g, 1, 1, 11, 3), _randn(g, 1, 1, 11, 2)
+    out = oracle.dca(qi, qs, qe, k, v, chunk=3, qk_scale=0.7, plant=plant)
+    ref = np.zeros_like(out)
+    for h in range(2):
+        for i in range(11):
+            w = []
+            for j in range(i + 1):
+                d = i // 3 - j // 3
+                qq = qi if d == 0 else (qs if d == 1 else qe)
+                w.append(math.exp(0.7 * sum(float(qq[0, h, i, t]) * float(k[0, 0, j, t]) for t in range(3))))
+            tot = sum(w)
+            for c in range(2):
+                ref[0, h, i, c] = sum(w[j] * float(v[0, 0, j, c]) for j in range(i + 1)) / tot
+    return _close(out, ref)
+
+
+DCA_PINS = [pin_dca_equal_queries_is_causal_attention, pin_dca_one_chunk_is_intra_only,
+            pin_dca_brute_force]
+
 # Planted mistakes compiled into copies of the oracle (ORACLE_PLANT=n).
 PLANTS = {
     1: "GQA group index h % kvHeadNum instead of h / (headNum / kvHeadNum)",

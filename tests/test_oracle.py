@@ -33,6 +33,17 @@ def test_merge_planted_mistake_is_caught(plant):
     assert failed, f"no pin catches planted merge mistake {plant}: {oracle.MERGE_PLANTS[plant]}"
 
 
+@pytest.mark.parametrize("pin", P.DCA_PINS, ids=lambda f: f.__name__)
+def test_dca_pin_holds(pin):
+    assert pin()
+
+
+@pytest.mark.parametrize("plant", sorted(oracle.DCA_PLANTS), ids=lambda n: oracle.DCA_PLANTS[n])
+def test_dca_planted_mistake_is_caught(plant):
+    failed = [p.__name__ for p in P.DCA_PINS if not p(plant)]
+    assert failed, f"no pin catches planted DCA mistake {plant}: {oracle.DCA_PLANTS[plant]}"
+
+
 def test_rows_mode_matches_full():
     g = torch.Generator().manual_seed(30)
     lens = torch.tensor([7, 3, 9], dtype=torch.int32)
