@@ -45,6 +45,7 @@ SIGNATURES = {
     "wf_attn_fwd_ex": (_I32, [_T, _T, _T, _T, _T, _T, _T, _T, _I32, _I32, _F32, _I32, _T, _T, _I32,
                               _P]),
     "wf_attn_merge": (_I32, [_T, _T, _T, _T, _P]),
+    "wf_attn_dca": (_I32, [_T, _T, _T, _T, _T, _I64, _I32, _I32, _F32, _T, _T, _P]),
     "wf_attn_fwd_debug": (_I32, [_T, _T, _T, _T, _T, _T, _T, _T, _I32, _I32, _F32, _I32, _T, _P,
                                  _U32, _I64]),
     "wf_attn_fwd_varlen_noalloc": (_I32, [_T, _T, _T, _T, _T, _T, _T, _I32, _I32, _F32, _I32, _T,

@@ -187,6 +187,27 @@ def merge(out_parts, lse_parts, *, out=None, lse=None, stream=None):
     return out, lse
 
 
+def dca(q_intra, q_succ, q_inter, k, v, chunk_size, *, qk_scale=None, out=None, return_lse=False,
+        stream=None):
+    """Dual chunk attention (``wf_attn_dca``): query i of chunk c attends
+    causally, scoring keys of chunk c with ``q_intra``, of chunk c - 1 with
+    ``q_succ`` and of earlier chunks with ``q_inter`` (each [B, H, L, D],
+    rotated by the caller for its position map); k / v [B, Hkv, L, D]."""
+    _require_cuda(q_intra, q_succ, q_inter, k, v, out)
+    if qk_scale is None:
+        qk_scale = 1.0 / math.sqrt(q_intra.shape[-1])
+    if out is None:
+        out = torch.empty(q_intra.shape[:3] + (v.shape[-1],), dtype=q_intra.dtype, device=q_intra.device)
+    lse = torch.empty(q_intra.shape[:3], dtype=torch.float32, device=q_intra.device) if return_lse else None
+    ds = [describe(x) for x in (q_intra, q_succ, q_inter, k, v)]
+    od, ld = describe(out), describe(lse)
+    with torch.cuda.device(q_intra.device):
+        _check(L.load().wf_attn_dca(*[ctypes.byref(d) for d in ds], int(chunk_size), int(q_intra.shape[1]),
+                                    int(k.shape[1]), float(qk_scale), ctypes.byref(od), _ref(ld),
+                                    _stream(stream)))
+    return (out, lse) if return_lse else out
+
+
 def device_status(stream=None) -> None:
     """Synchronize the stream and raise if a kernel recorded a device-side error."""
     _check(L.load().wf_get_device_status(_stream(stream)))

@@ -12,6 +12,7 @@
 //
 // One warp per row, four consecutive columns per lane per pass (128 columns
 // a pass); HBM-bound: it reads S partial rows and writes one.
+#include <algorithm>
 #include <cstdint>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -126,7 +127,19 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(const __grid_co
     mp.lse[i0 * mp.e_s0 + i1 * mp.e_s1 + i2 * mp.e_s2] = empty ? -INFINITY : top + __log2f(total) * kLn2M;
 }
 
+__global__ void fill_f32_kernel(float *dst, int64_t n, float v) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+    dst[i] = v;
+}
+
 }  // namespace
+
+cudaError_t launch_fill_f32(float *dst, int64_t n, float v, cudaStream_t stream) {
+  if (n <= 0) return cudaSuccess;
+  const int64_t blocks = std::min<int64_t>((n + 255) / 256, 148 * 8);
+  fill_f32_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(dst, n, v);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_merge(const MergeParams &mp, cudaStream_t stream) {
   if (mp.rows <= 0) return cudaSuccess;

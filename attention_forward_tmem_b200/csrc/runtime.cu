@@ -121,6 +121,33 @@ static wf_status_t stream_workspace(int dev, cudaStream_t stream, size_t bytes, 
   return WF_OK;
 }
 
+// Scratch of one (device, stream) for calls that run several attention calls
+// (dual chunk attention): separate from the workspace those calls use.
+static std::map<std::pair<int, cudaStream_t>, std::pair<void *, size_t>> g_scratch;
+
+wf_status_t stream_scratch(cudaStream_t stream, size_t bytes, void **out) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lock(g_mu);
+  auto &slot = g_scratch[{dev, stream}];
+  if (slot.second < bytes) {
+    if (slot.first) {
+      cudaError_t e = cudaStreamSynchronize(stream);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+      cudaFree(slot.first);
+      slot.first = nullptr;
+      slot.second = 0;
+    }
+    void *p = nullptr;
+    cudaError_t e = cudaMalloc(&p, bytes);
+    if (e != cudaSuccess) return fail(WF_ERR_NO_MEMORY, "cudaMalloc(%zu): %s", bytes, cudaGetErrorString(e));
+    slot.first = p;
+    slot.second = bytes;
+  }
+  *out = slot.first;
+  return WF_OK;
+}
+
 // ----------------------------------------------------------- TMA descriptors
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
@@ -210,6 +237,7 @@ constexpr int64_t kMinTilesPerSplit = 4;   // automatic split: KV tiles per spli
 static int32_t elem_type(int32_t dtype) {
   return dtype == WF_F32 ? kElemF32 : dtype == WF_F16 ? kElemF16 : kElemBF16;
 }
+int32_t elem_type_of(int32_t dtype) { return elem_type(dtype); }
 
 struct Dims {
   bool varlen, kv_padded;
@@ -729,6 +757,13 @@ void wf_shutdown(void) {
     }
   }
   g_workspaces.clear();
+  for (auto &kv : g_scratch) {
+    if (kv.second.first) {
+      cudaSetDevice(kv.first.first);
+      cudaFree(kv.second.first);
+    }
+  }
+  g_scratch.clear();
   cudaSetDevice(cur);
 }
 

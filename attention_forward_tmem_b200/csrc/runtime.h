@@ -42,6 +42,14 @@ wf_status_t attn_fwd_fused(const wf_tensor_t *q, const wf_tensor_t *k_view, cons
                            const wf_tensor_t *k_chunk, const wf_tensor_t *v_chunk, int64_t lo,
                            int64_t hi, int32_t headNum, int32_t kvHeadNum, float qkScale,
                            wf_tensor_t *out, void *stream, bool *declined);
+// Per-(device, stream) scratch for calls that compose several attention calls;
+// grown on demand (synchronizing the stream first), freed by wf_shutdown.
+wf_status_t stream_scratch(cudaStream_t stream, size_t bytes, void **out);
+// Element type code (ElemType) of a wf_dtype_t.
+int32_t elem_type_of(int32_t dtype);
+// Fill n floats with v (device, asynchronous).
+cudaError_t launch_fill_f32(float *dst, int64_t n, float v, cudaStream_t stream);
+
 // Zero the allocation-free entry's work-item counters on the current device
 // (noalloc.cu); used after a launch was aborted.
 cudaError_t reset_noalloc_counters();

@@ -205,6 +205,31 @@ wf_status_t wf_attn_merge(const wf_tensor_t *outParts, const wf_tensor_t *lsePar
                           wf_tensor_t *out, wf_tensor_t *lse, void *stream);
 
 /*
+ * wf_attn_dca -- dual chunk attention ("Dual Chunk Attention" article: a long
+ * sequence cut into chunks, attended within a chunk, to the neighbouring
+ * chunk and across chunks with remapped relative positions).  The article
+ * gives no formulas; the reading here: every query comes in three forms, the
+ * caller having rotated each for its position map, and query i of chunk
+ * c = i / chunkSize attends causally to keys j <= i with
+ *     qIntra (j in chunk c), qSucc (j in chunk c - 1), qInter (earlier chunks),
+ * all scores times qkScale in one softmax.
+ *   qIntra, qSucc, qInter: [B, headNum, L, D];  k: [B, kvHeadNum, L, D];
+ *   v: [B, kvHeadNum, L, Dv];  out: [B, headNum, L, Dv];  lse: NULL or
+ *   [B, headNum, L] WF_F32 (natural log).  WF_BF16 or WF_F16; D, Dv as for
+ *   wf_attn_fwd; strides as for its dense layout.
+ * Runs as three attention calls over disjoint key sets (causal within the
+ * chunks, chunk c against chunk c - 1, chunk c >= 2 against keys before
+ * chunk c - 1) and the merge pass; a library-owned per-stream scratch holds
+ * the three parts (3 L headNum (Dv x element size + 4) bytes).  Errors as
+ * wf_attn_fwd; asynchronous.
+ */
+wf_status_t wf_attn_dca(const wf_tensor_t *qIntra, const wf_tensor_t *qSucc,
+                        const wf_tensor_t *qInter, const wf_tensor_t *k,
+                        const wf_tensor_t *v, int64_t chunkSize, int32_t headNum,
+                        int32_t kvHeadNum, float qkScale, wf_tensor_t *out,
+                        wf_tensor_t *lse, void *stream);
+
+/*
  * wf_attn_fwd_debug -- wf_attn_fwd with test switches for the bounded waits
  * (no counterpart on the pages; a diagnostic aid).
  *   debug_flags bit 0: the kernel's copy engine never loads the first K tile,

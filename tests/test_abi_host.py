@@ -266,6 +266,34 @@ def test_merge_argument_errors(lib, case, expect):
         assert lib.wf_last_error_message()
 
 
+@pytest.mark.parametrize("case,expect", [
+    ("ok", None),
+    ("fp32", L.WF_ERR_UNSUPPORTED),
+    ("chunk_zero", L.WF_ERR_INVALID_ARG),
+    ("q_forms_differ", L.WF_ERR_INVALID_ARG),
+    ("kv_len", L.WF_ERR_INVALID_ARG),
+    ("out_shape", L.WF_ERR_INVALID_ARG),
+])
+def test_dca_argument_errors(lib, case, expect):
+    dt = L.WF_F32 if case == "fp32" else L.WF_BF16
+    qi, qs, qe = _t([1, 4, 300, 128], dt), _t([1, 4, 300, 128], dt), _t([1, 4, 300, 128], dt)
+    k, v, o = _t([1, 2, 300, 128], dt), _t([1, 2, 300, 128], dt), _t([1, 4, 300, 128], dt)
+    chunk = 0 if case == "chunk_zero" else 128
+    if case == "q_forms_differ":
+        qe = _t([1, 4, 299, 128], dt)
+    elif case == "kv_len":
+        k = _t([1, 2, 301, 128], dt)
+    elif case == "out_shape":
+        o = _t([1, 4, 300, 64], dt)
+    r = ctypes.byref
+    st = lib.wf_attn_dca(r(qi), r(qs), r(qe), r(k), r(v), chunk, 4, 2, 0.1, r(o), None, None)
+    if expect is None:
+        assert st in (L.WF_ERR_NO_DEVICE, L.WF_OK)
+    else:
+        assert st == expect
+        assert lib.wf_last_error_message()
+
+
 # ------------------------------------------------------------------ BlockKVCache
 
 def _cache(lib, L_=8, chunk=2, window=6, sink=2, seq_dim=2):
