@@ -73,6 +73,7 @@ extern "C" wf_status_t wf_attn_dca(const wf_tensor_t *qIntra, const wf_tensor_t 
   }
   if (B == 0 || L == 0) return WF_OK;
   if (Dv % 8 != 0) return fail(WF_ERR_UNSUPPORTED, "Dv must be a multiple of 8");
+  if (!current_device_state(&st)) return st;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
 
   // Scratch: 3 parts [L][H][Dv] (input type), their LSE [3][L][H] fp32, lengths.
