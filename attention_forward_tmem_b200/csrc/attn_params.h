@@ -90,8 +90,9 @@ struct AttnKernel {
   int32_t unit_rows;     // query rows per work unit of this kernel
 };
 
-// Kernel for (ElemType, dqk, drope, dv); launch == nullptr if none.
-AttnKernel find_attn_kernel(int dtype, int dqk, int drope, int dv);
+// Kernel for (ElemType, dqk, drope, dv), optionally the instance that also
+// writes a BlockKVCache chunk; launch == nullptr if none.
+AttnKernel find_attn_kernel(int dtype, int dqk, int drope, int dv, bool fused = false);
 
 // V [rows, heads, batch] x d (element strides) -> V^T [batch][heads][d][ld] (fp32).
 cudaError_t launch_transpose_v(const float *v, int64_t s_row, int64_t s_head, int64_t s_batch,

@@ -33,8 +33,12 @@ constexpr uint32_t kPPOtherRegs = 120;       // warpgroup 2: producer, MMA, 2 id
 // launch: 384 threads x 168 registers = 64512 >= 2*128*200 + 128*96 = 63488
 static_assert(2 * 128 * kPPSoftmaxRegs + 128 * kPPOtherRegs <= kPPThreads * 168, "register split");
 
-template <typename T, int DQK, int DROPE, int DV>
+// kFuse: the kernel instance that also writes a BlockKVCache chunk (key rows
+// [fuse_lo, fuse_hi) read from the chunk and stored into the cache); the
+// plain instance carries none of that code.
+template <typename T, int DQK, int DROPE, int DV, bool kFuse_ = false>
 struct PPCfg {
+  static constexpr bool kFuse = kFuse_;
   static constexpr int kAtomE = 64;                       // bf16 elements per 128-byte row
   static constexpr int kKStep = 16;
   static constexpr int kQAtoms = (DQK + kAtomE - 1) / kAtomE;
@@ -111,7 +115,7 @@ __device__ void pp_producer(const AttnParams &p, uint8_t *smem, PPCtrl *ctl, Pro
     tma_prefetch_map(&p.tm_qr);
     tma_prefetch_map(&p.tm_kr);
   }
-  if (p.fuse_hi > 0) {
+  if (Cfg::kFuse) {
     tma_prefetch_map(&p.tm_kc);
     tma_prefetch_map(&p.tm_vc);
   }
@@ -131,7 +135,7 @@ __device__ void pp_producer(const AttnParams &p, uint8_t *smem, PPCtrl *ctl, Pro
     }
     const int32_t krow = ti.krow + j * kBlockN;
     // rows of the new chunk (fused cache write) come from the chunk itself
-    const bool fz = krow >= p.fuse_lo && krow < p.fuse_hi;
+    const bool fz = Cfg::kFuse && krow >= p.fuse_lo && krow < p.fuse_hi;
     const CUtensorMap *mk = fz ? &p.tm_kc : &p.tm_k;
     const int32_t ry = fz ? krow - p.fuse_lo : krow;
     uint8_t *dst = smem + Cfg::kKOff + st * Cfg::kKBytes;
@@ -150,7 +154,7 @@ __device__ void pp_producer(const AttnParams &p, uint8_t *smem, PPCtrl *ctl, Pro
     const uint32_t gg = g + j, st = gg % Cfg::kVStages, n = gg / Cfg::kVStages;
     if (!bwait(&ctl->v_empty[st], (n + 1) & 1, &ctl->abort, p)) return false;
     const int32_t krow = ti.krow + j * kBlockN;
-    const bool fz = krow >= p.fuse_lo && krow < p.fuse_hi;
+    const bool fz = Cfg::kFuse && krow >= p.fuse_lo && krow < p.fuse_hi;
     const CUtensorMap *mv = fz ? &p.tm_vc : &p.tm_v;
     const int32_t ry = fz ? krow - p.fuse_lo : krow;
     uint8_t *dst = smem + Cfg::kVOff + st * Cfg::kVBytes;
@@ -269,6 +273,7 @@ __device__ void pp_mma(const AttnParams &p, uint8_t *smem, PPCtrl *ctl, uint32_t
   TileInfo ti0;
   bool writer = false, pending = false;
   auto store_tile = [&](bool is_k, uint32_t gg, int32_t jj) {
+    if constexpr (!Cfg::kFuse) return;
     const int32_t krow = ti0.krow + jj * kBlockN;
     if (!writer || krow < p.fuse_lo || krow >= p.fuse_hi) return;
     fence_proxy_async();
@@ -282,7 +287,7 @@ __device__ void pp_mma(const AttnParams &p, uint8_t *smem, PPCtrl *ctl, uint32_t
     pending = true;
   };
   auto stores_read = [&]() {
-    if (pending) {
+    if (Cfg::kFuse && pending) {
       bulk_wait_read();
       pending = false;
     }
@@ -305,7 +310,7 @@ __device__ void pp_mma(const AttnParams &p, uint8_t *smem, PPCtrl *ctl, uint32_t
     const int32_t n[2] = {ti0.n_kv, tile_info(p, t, 1).n_kv};
     const int32_t n_max = max(n[0], n[1]);
     if (n_max == 0) continue;
-    writer = p.fuse_hi > 0 && ti0.q0 == 0 && ti0.h % p.group == 0;
+    writer = Cfg::kFuse && ti0.q0 == 0 && ti0.h % p.group == 0;
     if (!(ok = bwait(&ctl->q_full, u & 1, &ctl->abort, p))) break;
     if (!(ok = wait_k(g))) break;
     tc_fence_after();
@@ -325,18 +330,24 @@ __device__ void pp_mma(const AttnParams &p, uint8_t *smem, PPCtrl *ctl, uint32_t
       store_tile(true, gk, j);
       if (!(ok = wait_v(gv))) break;
       store_tile(false, gv, j - 1);
-#pragma unroll
-      for (int s = 0; s < 2; ++s) {
-        if (j - 1 < n[s] && !(ok = do_pv(s, j - 1, n[s], gv))) break;
-        if (j < n[s]) {
-          pp_issue_s<Cfg>(tmem, qb[s], kbase(gk), s);
-          tc_commit(&ctl->s_full[s]);
-        }
+      if (j - 1 < n[0] && !(ok = do_pv(0, j - 1, n[0], gv))) break;
+      if (j < n[0]) {
+        pp_issue_s<Cfg>(tmem, qb[0], kbase(gk), 0);
+        tc_commit(&ctl->s_full[0]);
       }
-      if (!ok) break;
+      if (j - 1 < n[1] && !(ok = do_pv(1, j - 1, n[1], gv))) break;
       stores_read();
+      // With a single V stage (MLA tiles) V(j-1), now handed to both PVs, is
+      // released before S_B(j) is issued, so that the next V load starts one
+      // S product earlier (the commit still completes only once the PVs have);
+      // with two stages the extra commit on this path costs more than it buys.
+      if constexpr (Cfg::kVStages == 1) tc_commit(&ctl->v_empty[gv % Cfg::kVStages]);
+      if (j < n[1]) {
+        pp_issue_s<Cfg>(tmem, qb[1], kbase(gk), 1);
+        tc_commit(&ctl->s_full[1]);
+      }
       tc_commit(&ctl->k_empty[gk % Cfg::kKStages]);
-      tc_commit(&ctl->v_empty[gv % Cfg::kVStages]);
+      if constexpr (Cfg::kVStages != 1) tc_commit(&ctl->v_empty[gv % Cfg::kVStages]);
     }
     if (!ok) break;
     // All S products of this unit are issued: Q may be replaced once they finish.
@@ -355,7 +366,7 @@ __device__ void pp_mma(const AttnParams &p, uint8_t *smem, PPCtrl *ctl, uint32_t
     g += n_max;
     ++u;
   }
-  bulk_wait_all();                 // cache stores complete before the CTA ends
+  if constexpr (Cfg::kFuse) bulk_wait_all();   // cache stores complete before the CTA ends
   tc_commit(&ctl->drain);
   drain_wait(&ctl->drain, 0, p);
 }
@@ -415,9 +426,9 @@ __device__ void pp_softmax(const AttnParams &p, PPCtrl *ctl, uint32_t tmem, int 
 }
 
 // --------------------------------------------------------------------- kernel
-template <typename T, int DQK, int DROPE, int DV>
+template <typename T, int DQK, int DROPE, int DV, bool kFuse>
 __global__ void __launch_bounds__(kPPThreads, 1) attn_fwd_pp_kernel(const __grid_constant__ AttnParams p) {
-  using Cfg = PPCfg<T, DQK, DROPE, DV>;
+  using Cfg = PPCfg<T, DQK, DROPE, DV, kFuse>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
@@ -488,10 +499,10 @@ __global__ void __launch_bounds__(kPPThreads, 1) attn_fwd_pp_kernel(const __grid
   }
 }
 
-template <typename T, int DQK, int DROPE, int DV>
+template <typename T, int DQK, int DROPE, int DV, bool kFuse>
 cudaError_t launch_attn_pp(const AttnParams &p, int grid, cudaStream_t stream) {
-  using Cfg = PPCfg<T, DQK, DROPE, DV>;
-  auto kern = attn_fwd_pp_kernel<T, DQK, DROPE, DV>;
+  using Cfg = PPCfg<T, DQK, DROPE, DV, kFuse>;
+  auto kern = attn_fwd_pp_kernel<T, DQK, DROPE, DV, kFuse>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        Cfg::kSmemBytes);
   if (e != cudaSuccess) return e;

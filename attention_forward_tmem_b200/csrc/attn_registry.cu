@@ -10,12 +10,23 @@ namespace wf {
 
 template <typename T, int DQK, int DROPE, int DV>
 cudaError_t launch_attn(const AttnParams &p, int grid, cudaStream_t stream);
-template <typename T, int DQK, int DROPE, int DV>
+template <typename T, int DQK, int DROPE, int DV, bool kFuse>
 cudaError_t launch_attn_pp(const AttnParams &p, int grid, cudaStream_t stream);
 
-AttnKernel find_attn_kernel(int dtype, int dqk, int drope, int dv) {
+AttnKernel find_attn_kernel(int dtype, int dqk, int drope, int dv, bool fused) {
+  // kernels that also write a BlockKVCache chunk (head sizes 64 and 128)
+  if (fused) {
+#define WF_CASE_FUSED(T, TI, Q, V) \
+  if (dtype == TI && dqk == Q && drope == 0 && dv == V) return {&launch_attn_pp<T, Q, 0, V, true>, 2 * kBlockM};
+    WF_CASE_FUSED(__nv_bfloat16, kElemBF16, 64, 64)
+    WF_CASE_FUSED(__nv_bfloat16, kElemBF16, 128, 128)
+    WF_CASE_FUSED(__half, kElemF16, 64, 64)
+    WF_CASE_FUSED(__half, kElemF16, 128, 128)
+#undef WF_CASE_FUSED
+    return {nullptr, 0};
+  }
 #define WF_CASE_PP(T, TI, Q, R, V) \
-  if (dtype == TI && dqk == Q && drope == R && dv == V) return {&launch_attn_pp<T, Q, R, V>, 2 * kBlockM};
+  if (dtype == TI && dqk == Q && drope == R && dv == V) return {&launch_attn_pp<T, Q, R, V, false>, 2 * kBlockM};
 #define WF_CASE_PP16(Q, R, V) \
   WF_CASE_PP(__nv_bfloat16, kElemBF16, Q, R, V) \
   WF_CASE_PP(__half, kElemF16, Q, R, V)

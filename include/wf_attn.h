@@ -332,8 +332,9 @@ wf_status_t wf_kvcache_cached(wf_kvcache_t *cache, wf_tensor_t *k_view,
  *     wf_kvcache_cached views.
  * The attention kernel reads the chunk's keys and values from k / v directly
  * and stores them into the ring slot as it goes, so no separate copy runs.
- * That needs 16-bit buffers and a chunk size that is a multiple of 128;
- * otherwise the call runs the copy and then wf_attn_fwd (same results).
+ * That needs 16-bit buffers, head sizes 64 or 128 and a chunk size that is a
+ * multiple of 128; otherwise the call runs the copy and then wf_attn_fwd
+ * (same results).
  * Results and cache contents are bit-identical to the unfused calls.
  * WF_ERR_ORDER out of phase; argument errors as wf_kvcache_update /
  * wf_attn_fwd, with nothing written.  On success the cache is in the state
