@@ -83,3 +83,37 @@ def test_mla_varlen_prefill_full_size():
                                mask_kind="causal", qk_scale=w.qk_scale, head_num=1, kv_head_num=1)
         got = out_c[starts[rows[:, 0]] + rows[:, 2], h]
         compare(got, ref, torch.bfloat16, f"mla h{h}")
+
+
+def test_blockkv_rolling_fused_full_size():
+    """The rolling-cache workload as bench.py times it (fused chunk call, 12
+    heads, chunk 1024, sink 1024, window 7168, 16 chunks): outputs and cache
+    contents bit-identical to the separate calls after every chunk, and the
+    last chunk's sampled rows against the oracle over the logical cache."""
+    w = W.WORKLOADS["blockkv_rolling"]
+    c = W.BLOCKKV
+    L = c["sink_size"] + c["window_size"]
+    shape = (1, w.head_num, L, w.dqk)
+    mk = lambda: api.BlockKVCache.allocate(shape, shape, chunk_size=c["chunk_size"],
+                                           window_size=c["window_size"], sink_size=c["sink_size"],
+                                           device=DEV, dtype=w.dtype)
+    unf, fus = mk(), mk()
+    for i in range(c["n_chunks"]):
+        q, k, v = (t.to(DEV) for t in W.blockkv_chunk(i, w.head_num, c["chunk_size"], w.dqk, w.dtype))
+        unf.before_update(i)
+        unf.update(k, v)
+        out_u = api.attn_fwd(q, unf.cached_k(), unf.cached_v(), qk_scale=w.qk_scale)
+        unf.after_update(i)
+        fus.before_update(i)
+        out_f = fus.update_attend(k, v, q, qk_scale=w.qk_scale)
+        if i == c["n_chunks"] - 1:
+            ko, vo = fus.gather_logical()
+            rng = np.random.default_rng(7)
+            rows = np.array([(0, h, r) for h in (0, 5, 11)
+                             for r in sorted({0, 1, 127, 128, 1022, 1023} | set(rng.integers(0, 1024, 12).tolist()))])
+            ref = oracle.sdpa_rows(q.cpu(), ko.cpu(), vo.cpu(), rows, qk_scale=w.qk_scale)
+            compare(out_f[0, rows[:, 1], rows[:, 2]], ref, w.dtype, "rolling fused, last chunk")
+        fus.after_update(i)
+        api.device_status()
+        assert torch.equal(out_u, out_f), f"chunk {i}: outputs differ"
+        assert torch.equal(unf.k_buf, fus.k_buf) and torch.equal(unf.v_buf, fus.v_buf), f"chunk {i}: caches differ"
