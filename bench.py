@@ -214,7 +214,8 @@ class Workload:
 
     def step(self, dev=None, out=None):
         d = dev or self.dev
-        kw = dict(mask_type=self.api.MaskType.CAUSAL, qk_scale=self.w.qk_scale, out=out or self.out)
+        kw = dict(mask_type=self.api.MaskType.CAUSAL, qk_scale=self.w.qk_scale,
+                  out=self.out if out is None else out)
         if self.name == "mla_varlen_prefill":
             kw.update(qrope=d["qrope"], krope=d["krope"], q_seqlen=d["q_seqlen"],
                       kv_seqlen=d["kv_seqlen"])
@@ -377,28 +378,53 @@ def time_device(wl, steps, warmup, dist_on):
 
 
 def time_e2e(wl, steps, warmup):
-    """Same steps through the public API with host inputs: pinned host -> device
-    copies of q/k/v (+lengths) and the device -> host copy of the output are
-    inside the timed region."""
+    """Same steps through the public API with host inputs: every step copies
+    its q/k/v (+lengths) from pinned host memory to the device and reads its
+    output back, all inside the timed region.  As a server streaming requests
+    would, step i+1's uploads run on a second stream while step i computes and
+    its output is read back (device inputs and outputs double-buffered; events
+    order the buffer reuse), so the two copy directions and the compute
+    overlap."""
     pinned = {k: v.pin_memory() for k, v in wl.host.items()}
     out_host = torch.empty(wl.out.shape, dtype=wl.out.dtype).pin_memory()
-    dev = {k: torch.empty_like(v, device=wl.device) for k, v in pinned.items()}
-    stream = torch.cuda.current_stream()
+    dev = [{k: torch.empty_like(v, device=wl.device) for k, v in pinned.items()} for _ in range(2)]
+    outs = [torch.empty_like(wl.out) for _ in range(2)]
+    comp = torch.cuda.current_stream()
+    copy = torch.cuda.Stream()
+    loaded = [torch.cuda.Event() for _ in range(2)]
+    freed = [torch.cuda.Event() for _ in range(2)]
 
-    def one():
-        for k in pinned:
-            dev[k].copy_(pinned[k], non_blocking=True)
-        wl.step(dev=dev)
-        out_host.copy_(wl.out, non_blocking=True)
+    def upload(i):
+        b = i % 2
+        copy.wait_event(freed[b])          # step i-2 has finished reading these buffers
+        with torch.cuda.stream(copy):
+            for k in pinned:
+                dev[b][k].copy_(pinned[k], non_blocking=True)
+            loaded[b].record(copy)
 
-    for _ in range(warmup):
-        one()
+    def compute(i):
+        b = i % 2
+        comp.wait_event(loaded[b])
+        wl.step(dev=dev[b], out=outs[b])
+        freed[b].record(comp)
+        out_host.copy_(outs[b], non_blocking=True)
+
+    def run(n, start):
+        copy.wait_event(start)
+        upload(0)
+        for i in range(n):
+            if i + 1 < n:
+                upload(i + 1)
+            compute(i)
+
+    e_w = torch.cuda.Event()
+    e_w.record(comp)
+    run(warmup, e_w)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(steps):
-        one()
-    e1.record(stream)
+    e0.record(comp)
+    run(steps, e0)
+    e1.record(comp)
     torch.cuda.synchronize()
     h2d = sum(t.numel() * t.element_size() for t in pinned.values())
     d2h = out_host.numel() * out_host.element_size()
