@@ -332,6 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
+  pdl_wait();                       // the previous launch's results are visible from here on
 
   ProducerLog plog;
   if (warp < 4) {
@@ -341,6 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   } else {
     if ((threadIdx.x & 31) == 0) mma_role<Cfg>(p, smem, ctl, tmem);
   }
+  pdl_trigger();
 
   tc_fence_before();
   __syncthreads();
@@ -360,8 +362,7 @@ cudaError_t launch_attn(const AttnParams &p, int grid, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        Cfg::kSmemBytes);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, Cfg::kSmemBytes, stream>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3(kThreads), Cfg::kSmemBytes, stream, p);
 }
 
 }  // namespace wf

@@ -85,6 +85,26 @@ struct alignas(64) AttnParams {
 
 using AttnLaunchFn = cudaError_t (*)(const AttnParams &, int grid, cudaStream_t);
 
+// Launch with programmatic stream serialization: the kernel may begin (its
+// prologue) while the previous launch on the stream finishes; every kernel of
+// the library waits (pdl_wait) before it touches global memory, and signals
+// (pdl_trigger) once its own work is done.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 struct AttnKernel {
   AttnLaunchFn launch;
   int32_t unit_rows;     // query rows per work unit of this kernel

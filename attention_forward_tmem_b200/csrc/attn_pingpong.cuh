@@ -466,6 +466,7 @@ __global__ void __launch_bounds__(kPPThreads, 1) attn_fwd_pp_kernel(const __grid
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
+  pdl_wait();                       // the previous launch's results are visible from here on
 
   ProducerLog plog;
   if (warp < 8) {
@@ -476,6 +477,7 @@ __global__ void __launch_bounds__(kPPThreads, 1) attn_fwd_pp_kernel(const __grid
     if (warp == 8 && (threadIdx.x & 31) == 0) pp_producer<Cfg>(p, smem, ctl, plog);
     if (warp == 9 && (threadIdx.x & 31) == 0) pp_mma<Cfg>(p, smem, ctl, tmem);
   }
+  pdl_trigger();
 
   tc_fence_before();
   __syncthreads();
@@ -506,8 +508,7 @@ cudaError_t launch_attn_pp(const AttnParams &p, int grid, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        Cfg::kSmemBytes);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kPPThreads, Cfg::kSmemBytes, stream>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3(kPPThreads), Cfg::kSmemBytes, stream, p);
 }
 
 }  // namespace wf

@@ -16,7 +16,9 @@
 #include <cstring>
 #include <new>
 
+#include "attn_params.h"
 #include "runtime.h"
+#include "sm100_ptx.cuh"
 
 using namespace wf;
 
@@ -71,6 +73,8 @@ __global__ void copy_rows_kernel(const uint8_t *__restrict__ src, int64_t s_b, i
                                  int64_t s_t, uint8_t *__restrict__ dst, int64_t d_b, int64_t d_h,
                                  int64_t d_t, int64_t dst_t0, int64_t H, int64_t C, int64_t n_rows,
                                  int64_t units_per_row) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t total = n_rows * units_per_row;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
        i += (int64_t)gridDim.x * blockDim.x) {
@@ -112,14 +116,14 @@ wf_status_t copy_positions(const void *src_base, const View &s, int64_t src_t0, 
   if (blocks > 148 * 16) blocks = 148 * 16;
   const int64_t sb = s.sb * es, sh = s.sh * es, st = s.sl * es;
   const int64_t db = d.sb * es, dh = d.sh * es, dt = d.sl * es;
+  cudaError_t e;
   switch (unit) {
-    case 16: copy_rows_kernel<uint4><<<(int)blocks, threads, 0, stream>>>(src, sb, sh, st, dst, db, dh, dt, dst_t0, s.H, C, rows, upr); break;
-    case 8: copy_rows_kernel<uint2><<<(int)blocks, threads, 0, stream>>>(src, sb, sh, st, dst, db, dh, dt, dst_t0, s.H, C, rows, upr); break;
-    case 4: copy_rows_kernel<uint32_t><<<(int)blocks, threads, 0, stream>>>(src, sb, sh, st, dst, db, dh, dt, dst_t0, s.H, C, rows, upr); break;
-    case 2: copy_rows_kernel<uint16_t><<<(int)blocks, threads, 0, stream>>>(src, sb, sh, st, dst, db, dh, dt, dst_t0, s.H, C, rows, upr); break;
-    default: copy_rows_kernel<uint8_t><<<(int)blocks, threads, 0, stream>>>(src, sb, sh, st, dst, db, dh, dt, dst_t0, s.H, C, rows, upr); break;
+    case 16: e = launch_pdl(copy_rows_kernel<uint4>, dim3((unsigned)blocks), dim3(threads), 0, stream, src, sb, sh, st, dst, db, dh, dt, dst_t0, s.H, C, rows, upr); break;
+    case 8: e = launch_pdl(copy_rows_kernel<uint2>, dim3((unsigned)blocks), dim3(threads), 0, stream, src, sb, sh, st, dst, db, dh, dt, dst_t0, s.H, C, rows, upr); break;
+    case 4: e = launch_pdl(copy_rows_kernel<uint32_t>, dim3((unsigned)blocks), dim3(threads), 0, stream, src, sb, sh, st, dst, db, dh, dt, dst_t0, s.H, C, rows, upr); break;
+    case 2: e = launch_pdl(copy_rows_kernel<uint16_t>, dim3((unsigned)blocks), dim3(threads), 0, stream, src, sb, sh, st, dst, db, dh, dt, dst_t0, s.H, C, rows, upr); break;
+    default: e = launch_pdl(copy_rows_kernel<uint8_t>, dim3((unsigned)blocks), dim3(threads), 0, stream, src, sb, sh, st, dst, db, dh, dt, dst_t0, s.H, C, rows, upr); break;
   }
-  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "cache copy launch");
   return WF_OK;
 }

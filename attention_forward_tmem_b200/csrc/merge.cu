@@ -62,6 +62,8 @@ __device__ __forceinline__ void store4(void *base, int64_t idx, int32_t type, co
 }
 
 __global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(const __grid_constant__ MergeParams mp) {
+  pdl_wait();                        // the partial rows of the previous launch
+  pdl_trigger();
   int64_t rows = mp.rows;
   if (mp.sched) {
     if (mp.sched[1] != 0) return;                                   // lengths were rejected
@@ -128,6 +130,8 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(const __grid_co
 }
 
 __global__ void fill_f32_kernel(float *dst, int64_t n, float v) {
+  pdl_wait();
+  pdl_trigger();
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
     dst[i] = v;
 }
@@ -137,16 +141,14 @@ __global__ void fill_f32_kernel(float *dst, int64_t n, float v) {
 cudaError_t launch_fill_f32(float *dst, int64_t n, float v, cudaStream_t stream) {
   if (n <= 0) return cudaSuccess;
   const int64_t blocks = std::min<int64_t>((n + 255) / 256, 148 * 8);
-  fill_f32_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(dst, n, v);
-  return cudaGetLastError();
+  return launch_pdl(fill_f32_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, stream, dst, n, v);
 }
 
 cudaError_t launch_merge(const MergeParams &mp, cudaStream_t stream) {
   if (mp.rows <= 0) return cudaSuccess;
   const int64_t blocks = (mp.rows + kMergeWarps - 1) / kMergeWarps;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  merge_kernel<<<static_cast<unsigned>(blocks), kMergeWarps * 32, 0, stream>>>(mp);
-  return cudaGetLastError();
+  return launch_pdl(merge_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kMergeWarps * 32), 0, stream, mp);
 }
 
 }  // namespace wf

@@ -13,6 +13,7 @@
 #include <cstdint>
 
 #include "attn_params.h"
+#include "sm100_ptx.cuh"
 
 namespace wf {
 namespace {
@@ -59,6 +60,8 @@ __global__ void __launch_bounds__(kSchedThreads) sched_prep_kernel(
   __shared__ int32_t bad;
   __shared__ int64_t carry_q, carry_k, carry_w;
   const int tid = threadIdx.x;
+  pdl_wait();
+  pdl_trigger();
   if (tid == 0) {
     bad = 0;
     carry_q = carry_k = carry_w = 0;
@@ -163,9 +166,8 @@ cudaError_t launch_sched_prep(const int32_t *q_len, const int32_t *k_len, int32_
                               int32_t head_num, int32_t unit_rows, int32_t *ws,
                               const SchedLayout &sl, int32_t *status, cudaStream_t stream) {
   static_assert(kHistBins == 4 * kSchedThreads, "scan covers 4 bins per thread");
-  sched_prep_kernel<<<1, kSchedThreads, 0, stream>>>(q_len, k_len, batch, n_q_tokens, n_k_tokens,
-                                                     k_max_len, head_num, ws, unit_rows, sl, status);
-  return cudaGetLastError();
+  return launch_pdl(sched_prep_kernel, dim3(1), dim3(kSchedThreads), 0, stream, q_len, k_len, batch,
+                    n_q_tokens, n_k_tokens, k_max_len, head_num, ws, unit_rows, sl, status);
 }
 
 }  // namespace wf
