@@ -224,3 +224,27 @@ def test_repeated_calls_are_deterministic():
     b = api.attn_fwd(qd, kd, vd, mask_type=api.MaskType.CAUSAL)
     api.device_status()
     assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("kind", ["none", "causal"])
+def test_dense_without_keys_gives_zero_rows(dtype, kind):
+    """Lk = 0: every row sees no key, so it is 0 with LSE -inf (the silent case's reading)."""
+    q = torch.randn(1, 4, 200, 128).to(dtype).to(DEV)
+    k = torch.empty(1, 2, 0, 128, dtype=dtype, device=DEV)
+    v = torch.empty(1, 2, 0, 128, dtype=dtype, device=DEV)
+    mt = api.MaskType.CAUSAL if kind == "causal" else api.MaskType.NONE
+    out, lse = api.attn_fwd(q, k, v, mask_type=mt, return_lse=True)
+    api.device_status()
+    assert torch.all(out == 0) and torch.all(torch.isneginf(lse))
+
+
+def test_packed_without_keys_gives_zero_rows():
+    ql = torch.tensor([30, 0, 70], dtype=torch.int32)
+    kl = torch.tensor([0, 0, 0], dtype=torch.int32)
+    q = torch.randn(100, 2, 128).to(torch.bfloat16).to(DEV)
+    k = torch.empty(0, 2, 128, dtype=torch.bfloat16, device=DEV)
+    out = torch.full((100, 2, 128), 3.0, dtype=torch.bfloat16, device=DEV)
+    out, lse = api.attn_fwd(q, k, k, q_seqlen=ql.to(DEV), kv_seqlen=kl.to(DEV), out=out, return_lse=True)
+    api.device_status()
+    assert torch.all(out == 0) and torch.all(torch.isneginf(lse))
