@@ -262,7 +262,20 @@ __device__ __forceinline__ void store_row(const AttnParams &p, const TileInfo &t
                                           const float (&o)[DV], float inv) {
   T *dst = reinterpret_cast<T *>(p.out) + (int64_t)ti.b * p.o_sb + (int64_t)ti.h * p.o_sh +
            (int64_t)(p.varlen ? ti.qrow + (row - ti.q0) : row) * p.o_si;
+  // One thread writes one row, so every store instruction of a warp touches
+  // 32 rows; 32-byte stores halve the instructions and the cache-line visits
+  // against 16-byte ones (rows whose start is not 32-byte aligned take those).
   if constexpr (sizeof(T) == 2) {
+    if (DV % 16 == 0 && (reinterpret_cast<uintptr_t>(dst) & 31) == 0) {
+#pragma unroll
+      for (int c = 0; c < DV; c += 16) {
+        uint32_t w[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) w[i] = Elem16<T>::pack2(o[c + 2 * i] * inv, o[c + 2 * i + 1] * inv);
+        st_global_v8(dst + c, w);
+      }
+      return;
+    }
 #pragma unroll
     for (int c = 0; c < DV; c += 8) {
       uint4 v;
@@ -273,6 +286,16 @@ __device__ __forceinline__ void store_row(const AttnParams &p, const TileInfo &t
       *reinterpret_cast<uint4 *>(dst + c) = v;
     }
   } else {
+    if (DV % 8 == 0 && (reinterpret_cast<uintptr_t>(dst) & 31) == 0) {
+#pragma unroll
+      for (int c = 0; c < DV; c += 8) {
+        uint32_t w[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) w[i] = __float_as_uint(o[c + i] * inv);
+        st_global_v8(dst + c, w);
+      }
+      return;
+    }
 #pragma unroll
     for (int c = 0; c < DV; c += 4) {
       float4 v = make_float4(o[c] * inv, o[c + 1] * inv, o[c + 2] * inv, o[c + 3] * inv);
@@ -294,11 +317,14 @@ __device__ __forceinline__ void store_result(const AttnParams &p, const TileInfo
     const int64_t r = p.varlen ? (int64_t)(ti.qrow - ti.q0 + row) * p.hq + ti.h
                                : ((int64_t)ti.b * p.hq + ti.h) * p.lq + row;
     const int64_t idx = (int64_t)ti.sp * p.part_rows + r;
-    float *dst = p.part_o + idx * DV;
+    float *dst = p.part_o + idx * DV;       // 256-byte aligned buffer, DV % 8 == 0
 #pragma unroll
-    for (int c = 0; c < DV; c += 4)
-      *reinterpret_cast<float4 *>(dst + c) =
-          make_float4(o[c] * inv, o[c + 1] * inv, o[c + 2] * inv, o[c + 3] * inv);
+    for (int c = 0; c < DV; c += 8) {
+      uint32_t w[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) w[i] = __float_as_uint(o[c + i] * inv);
+      st_global_v8(dst + c, w);
+    }
     p.part_lse[idx] = lse;
   } else {
     store_row<T, DV>(p, ti, row, o, inv);

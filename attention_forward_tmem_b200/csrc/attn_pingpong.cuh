@@ -83,23 +83,37 @@ struct PPCtrl {
   volatile int32_t sched_item[2];
   uint32_t tmem_base;
   volatile int32_t abort;
+  TileInfo sched_ti[2][2];        // both sub-tiles of the item in each ring slot
 };
+static_assert(sizeof(PPCtrl) <= 1024, "control block");
 
 // Work items are handed out at run time: the producer thread takes the next
-// item index from a global counter (atomicAdd) and publishes it in a two-slot
-// ring; the MMA thread and the 8 softmax warps read it from there.  Items
+// item index from a global counter (atomicAdd) and publishes it, with the
+// decoded tile coordinates of both sub-tiles, in a two-slot ring; the MMA
+// thread and the 8 softmax warps read it from there.  Decoding an item takes
+// integer divisions (and, for packed sequences, a search over the work prefix
+// sums); done once by the producer, which runs ahead, it stays off the path
+// from one item's last PV to the next item's first S.  Items
 // are thus processed in their enumeration order (locality first, longest
 // unit first) by whichever CTA is free, which keeps the K/V tensors in use at
 // one time few and balances the load.  The last CTA to exit resets the
 // counters for the next launch on the stream.
 constexpr uint32_t kSchedConsumers = 1 + 8;     // MMA thread + one lane per softmax warp
 
-// Consumer side: the next item (or a value >= the item count at the end).
+// Consumer side: the next item (or a value >= the item count at the end) and
+// the tile coordinates of sub-tile `sub` (both sub-tiles when sub < 0: ti[0],
+// ti[1]; meaningless past the last item).
 __device__ __forceinline__ bool pp_next_item(const AttnParams &p, PPCtrl *ctl, uint32_t &it,
-                                             int32_t &t, bool arrive) {
+                                             int32_t &t, TileInfo *ti, int sub, bool arrive) {
   const uint32_t k = it & 1;
   if (!bwait(&ctl->sched_full[k], (it >> 1) & 1, &ctl->abort, p)) return false;
   t = ctl->sched_item[k];
+  if (sub < 0) {
+    ti[0] = ctl->sched_ti[k][0];
+    ti[1] = ctl->sched_ti[k][1];
+  } else {
+    ti[0] = ctl->sched_ti[k][sub];
+  }
   if (arrive) mbar_arrive(&ctl->sched_empty[k]);
   ++it;
   return true;
@@ -172,9 +186,15 @@ __device__ void pp_producer(const AttnParams &p, uint8_t *smem, PPCtrl *ctl, Pro
     if (!(ok = bwait(&ctl->sched_empty[k], ((it >> 1) + 1) & 1, &ctl->abort, p))) break;
     const int32_t t = atomicAdd(p.counters, 1);
     ctl->sched_item[k] = t;
+    TileInfo t0, t1;
+    if (t < n_units) {
+      t0 = tile_info(p, t, 0);
+      t1 = tile_info(p, t, 1);
+      ctl->sched_ti[k][0] = t0;
+      ctl->sched_ti[k][1] = t1;
+    }
     mbar_arrive(&ctl->sched_full[k]);
     if (t >= n_units) break;
-    const TileInfo t0 = tile_info(p, t, 0), t1 = tile_info(p, t, 1);
     const int32_t n_max = max(t0.n_kv, t1.n_kv);
     if (n_max == 0) continue;
     if (!(ok = bwait(&ctl->q_empty, (u + 1) & 1, &ctl->abort, p))) break;
@@ -305,9 +325,10 @@ __device__ void pp_mma(const AttnParams &p, uint8_t *smem, PPCtrl *ctl, uint32_t
 
   for (uint32_t it = 0;;) {
     int32_t t;
-    if (!(ok = pp_next_item(p, ctl, it, t, true)) || t >= n_units) break;
-    ti0 = tile_info(p, t, 0);
-    const int32_t n[2] = {ti0.n_kv, tile_info(p, t, 1).n_kv};
+    TileInfo tis[2];
+    if (!(ok = pp_next_item(p, ctl, it, t, tis, -1, true)) || t >= n_units) break;
+    ti0 = tis[0];
+    const int32_t n[2] = {tis[0].n_kv, tis[1].n_kv};
     const int32_t n_max = max(n[0], n[1]);
     if (n_max == 0) continue;
     writer = Cfg::kFuse && ti0.q0 == 0 && ti0.h % p.group == 0;
@@ -384,11 +405,11 @@ __device__ void pp_softmax(const AttnParams &p, PPCtrl *ctl, uint32_t tmem, int 
   bool ok = true;
   for (uint32_t it = 0;;) {
     int32_t t;
-    ok = pp_next_item(p, ctl, it, t, false);
+    TileInfo ti;
+    ok = pp_next_item(p, ctl, it, t, &ti, s, false);
     __syncwarp();
     if (lane == 0 && ok) mbar_arrive(&ctl->sched_empty[(it - 1) & 1]);
     if (!ok || t >= n_units) break;
-    const TileInfo ti = tile_info(p, t, s);
     const int32_t row = ti.q0 + r;
     const bool row_valid = row < ti.lq;
     if (ti.n_kv == 0) {

@@ -64,6 +64,13 @@ __device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, u
       : "memory");
 }
 
+// 32-byte global store (sm_100 256-bit vector form); `ptr` 32-byte aligned.
+__device__ __forceinline__ void st_global_v8(void *ptr, const uint32_t (&w)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(ptr), "r"(w[0]),
+               "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
+}
+
 // TMA 4-d tiled store shared -> global (bulk async-group).  Coordinates are
 // never negative here, and c0 is a multiple of 16 bytes' worth of elements.
 __device__ __forceinline__ void tma_store_4d(const CUtensorMap *map, const void *src, int32_t c0,
