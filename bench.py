@@ -504,9 +504,10 @@ def _oracle_rows_rolling(w, rng, seed):
     return make, 2 * (w.dqk + w.dv) * mean_vis, desc
 
 
-def oracle_sample(name, budget_s=12.0, seed=7):
+def oracle_sample(name, budget_s=12.0, seed=7, n=None):
     """Time the fp64 oracle on rows of the workload (each over its full key
-    range) for about `budget_s` seconds.  Returns (TFLOP/s, threads, note)."""
+    range) for about `budget_s` seconds, or on `n` rows when given (no
+    calibration).  Returns (TFLOP/s, threads, note, rows)."""
     import oracle
     w = W.WORKLOADS[name]
     rng = np.random.default_rng(seed)
@@ -520,14 +521,25 @@ def oracle_sample(name, budget_s=12.0, seed=7):
         fn()
         return fl, time.perf_counter() - t0
 
-    n = 64
-    for share in (0.02, 0.15):                  # calibrate twice, then the timed sample
+    # Calibrate until a run takes a quarter of the budget (small runs are
+    # dominated by per-call overhead and overstate the cost of a row), then
+    # size the timed sample from that rate.
+    n_max = 400000
+    if n is not None:
         fl, dt = run(n)
-        n = int(min(400000, max(64, fl / max(dt, 1e-6) * budget_s * share / per_row)))
-    n = int(min(400000, max(64, fl / max(dt, 1e-6) * budget_s / per_row)))
-    fl, dt = run(n)
+    else:
+        n = 64
+        while True:
+            fl, dt = run(n)
+            if dt >= 0.25 * budget_s or n >= n_max:
+                break
+            n = int(min(n_max, max(2 * n, fl / max(dt, 1e-6) * budget_s * 0.3 / per_row)))
+        n_final = int(min(n_max, max(n, fl / max(dt, 1e-6) * budget_s / per_row)))
+        if n_final != n:
+            n = n_final
+            fl, dt = run(n)
     note = f"{n} query rows of {name} ({desc}), fp64 oracle, {dt:.1f} s"
-    return fl / dt / 1e12, oracle.oracle_threads(), note
+    return fl / dt / 1e12, oracle.oracle_threads(), note, n
 
 
 # -------------------------------------------------------------------- main
@@ -550,10 +562,15 @@ def reference_arm(args, rank, world):
     if rank != 0:
         return
     name = args.workload
+    # Each step is a bounded sample sized so that warm-up plus timed steps
+    # take about --ref-total-s seconds (at most 3 s a step): the row count is
+    # calibrated on the first warm-up step and kept, with fresh rows per step.
+    n_total = args.warmup + args.steps
+    step_s = args.ref_step_s if args.ref_step_s > 0 else min(3.0, max(0.05, args.ref_total_s / n_total))
     per_step = []
-    note = threads = None
-    for i in range(args.warmup + args.steps):
-        v, threads, note = oracle_sample(name, budget_s=args.ref_step_s, seed=100 + i)
+    note = threads = rows = None
+    for i in range(n_total):
+        v, threads, note, rows = oracle_sample(name, budget_s=step_s, seed=100 + i, n=rows)
         if i >= args.warmup:
             per_step.append(v)
     val = statistics.mean(per_step)
@@ -579,7 +596,10 @@ def main():
                              "blockkv_rolling"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--ref-step-s", type=float, default=3.0)
+    ap.add_argument("--ref-step-s", type=float, default=0.0,
+                    help="reference arm: seconds of oracle work per step (0: from --ref-total-s)")
+    ap.add_argument("--ref-total-s", type=float, default=150.0,
+                    help="reference arm: target seconds for warm-up plus timed steps")
     ap.add_argument("--no-extras", action="store_true",
                     help="time the product step only (no e2e, CPU baseline or comparison loop; for profilers)")
     args = ap.parse_args()
@@ -644,7 +664,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.no_extras:
-        v, threads, note = oracle_sample(args.workload)
+        v, threads, note, _ = oracle_sample(args.workload)
         cpu = {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": note}
 
     if dist_on:
