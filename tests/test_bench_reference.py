@@ -1,0 +1,48 @@
+"""bench.py's reference arm (the fp64 oracle on the host cores): one JSON line
+with the product arm's metric and unit, a bounded sample per step, rank 0
+only; and the warm-up floor of the timing rules."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _bench(args, env=None):
+    return subprocess.run([sys.executable, "bench.py", *args], cwd=ROOT, capture_output=True, text=True,
+                          timeout=600, env=env)
+
+
+@pytest.mark.parametrize("workload", ["gqa_causal_prefill", "blockkv_rolling"])
+def test_reference_arm_prints_one_json_line(workload):
+    r = _bench(["--impl", "reference", "--steps", "2", "--warmup", "3", "--ref-total-s", "2",
+                "--workload", workload])
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference"
+    assert d["unit"] == "TFLOP/s" and d["higher_is_better"] is True
+    assert d["steps"] == 2 and d["warmup"] == 3 and d["n_gpus"] == 1
+    assert d["value"] > 0
+    assert d["config"]["workload"] == workload
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_runs_on_rank_zero_only():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2")
+    r = _bench(["--impl", "reference", "--steps", "1", "--warmup", "3", "--ref-total-s", "1"], env=env)
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert r.stdout.strip() == ""
+
+
+def test_fewer_than_three_warmup_steps_are_rejected():
+    r = _bench(["--impl", "reference", "--steps", "1", "--warmup", "2"])
+    assert r.returncode != 0
+    assert "warmup" in r.stderr
