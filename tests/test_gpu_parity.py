@@ -122,6 +122,20 @@ def test_packed(cfg):
     compare(out, ref, torch.bfloat16, str(cfg))
 
 
+@pytest.mark.parametrize("causal", [True, False])
+def test_packed_many_sequences(causal):
+    """64 sequences of seeded random lengths in [0, 300] (kv lengths at least
+    the query lengths): many more work items than CTAs, so every CTA takes
+    several items through the scheduling ring, with empty sequences and
+    items whose second tile is empty among them."""
+    rng = np.random.default_rng(31)
+    ql = rng.integers(0, 301, 64)
+    ql[[3, 17, 40]] = 0
+    kl = ql + rng.integers(0, 60, 64)
+    out, ref = _run_packed(ql.tolist(), kl.tolist(), 8, 2, 128, 128, 0, causal, seed=32)
+    compare(out, ref, torch.bfloat16, f"64 sequences causal={causal}")
+
+
 @pytest.mark.parametrize("kind,mdtype,bshape", [
     ("keep", torch.bool, "full"), ("keep", torch.bool, "bcast"),
     ("add", torch.float32, "full"), ("add", torch.bfloat16, "full"), ("add", torch.float32, "bcast"),
