@@ -297,26 +297,38 @@ wf_status_t wf_attn_fwd_varlen_noalloc(const wf_tensor_t *q, const wf_tensor_t *
  * ------------------------------------------------------------------------- */
 typedef struct wf_kvcache wf_kvcache_t;
 
-/* Create a handle over caller-owned buffers (4-d, same dtype, last dim
- * contiguous).  No device memory is touched.  *out receives the handle. */
+/* Create a handle over caller-owned buffers (4-d, same dtype and shape apart
+ * from the last dim, last dim contiguous).  No device memory is touched.
+ * *out receives the handle, owned by the caller until wf_kvcache_destroy; the
+ * buffers must outlive it.  WF_ERR_INVALID_ARG for NULL or malformed buffers,
+ * seq_dim other than 1 or 2, sink_size + window_size different from the
+ * buffers' length L, L or sink_size not a multiple of chunk_size, or
+ * window_size < chunk_size; WF_ERR_NO_MEMORY if the host allocation fails. */
 wf_status_t wf_kvcache_create(const wf_tensor_t *k_buf, const wf_tensor_t *v_buf,
                               int32_t seq_dim, int64_t chunk_size,
                               int64_t sink_size, int64_t window_size,
                               wf_kvcache_t **out);
 
-/* Start chunk `chunk_idx` (host only, no device work). */
+/* Start chunk `chunk_idx` (host only, no device work).  WF_ERR_ORDER while a
+ * chunk is in progress or for an index the order rule above does not allow;
+ * the state is then unchanged. */
 wf_status_t wf_kvcache_before_update(wf_kvcache_t *cache, int64_t chunk_idx);
 
 /* Write the current chunk: k / v have the buffers' shape with exactly
- * chunk_size positions along seq_dim; copied on `stream` into the chunk's
- * slot. */
+ * chunk_size positions along seq_dim (same dtype, last dim contiguous);
+ * copied on `stream` into the chunk's slot (asynchronous; k / v must stay
+ * valid until the copy has run).  WF_ERR_ORDER unless before_update was the
+ * last call, WF_ERR_INVALID_ARG for a shape or dtype mismatch: nothing is
+ * written and the state is unchanged.  WF_ERR_CUDA if a copy cannot be
+ * launched (the K copy may have been issued when the V copy fails). */
 wf_status_t wf_kvcache_update(wf_kvcache_t *cache, const wf_tensor_t *k,
                               const wf_tensor_t *v, void *stream);
 
 /* Views of the visible prefix, returned in the logical [B, H, vis, D] form
- * (strides of the buffers), ready to pass to wf_attn_fwd as k / v.  Physical
- * ring order: attention without a causal mask does not depend on key order.
- * Host only. */
+ * (strides of the buffers; the data pointers point into the caller's
+ * buffers), ready to pass to wf_attn_fwd as k / v.  Physical ring order:
+ * attention without a causal mask does not depend on key order.  Host only.
+ * WF_ERR_ORDER before the chunk's update; either view pointer may be NULL. */
 wf_status_t wf_kvcache_cached(wf_kvcache_t *cache, wf_tensor_t *k_view,
                               wf_tensor_t *v_view, int64_t *visible_len);
 
@@ -344,7 +356,9 @@ wf_status_t wf_kvcache_update_attend(wf_kvcache_t *cache, const wf_tensor_t *k,
                                      int32_t headNum, float qkScale, wf_tensor_t *out,
                                      void *stream);
 
-/* Commit chunk `chunk_idx` (must equal the one in progress). Host only. */
+/* Commit chunk `chunk_idx` (must equal the one in progress). Host only.
+ * WF_ERR_ORDER before the cached views were taken (or the fused call ran) or
+ * for another index; the state is then unchanged. */
 wf_status_t wf_kvcache_after_update(wf_kvcache_t *cache, int64_t chunk_idx);
 
 /* Read the state: index in progress (-1 before the first), last committed
@@ -361,6 +375,8 @@ wf_status_t wf_kvcache_get_state(const wf_kvcache_t *cache, int64_t *cur_idx,
 wf_status_t wf_kvcache_gather_logical(wf_kvcache_t *cache, wf_tensor_t *k_out,
                                       wf_tensor_t *v_out, void *stream);
 
+/* Free the handle (host memory only; the buffers stay the caller's).
+ * NULL is ignored. */
 void wf_kvcache_destroy(wf_kvcache_t *cache);
 
 /* ---------------------------------------------------------------------------
