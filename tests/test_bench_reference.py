@@ -3,6 +3,7 @@ with the product arm's metric and unit, a bounded sample per step, rank 0
 only; and the warm-up floor of the timing rules."""
 import json
 import os
+import socket
 import subprocess
 import sys
 
@@ -40,6 +41,23 @@ def test_reference_arm_runs_on_rank_zero_only():
     r = _bench(["--impl", "reference", "--steps", "1", "--warmup", "3", "--ref-total-s", "1"], env=env)
     assert r.returncode == 0, r.stderr[-2000:]
     assert r.stdout.strip() == ""
+
+
+def test_reference_arm_under_torchrun_two_ranks():
+    """Launched as for N > 1: one JSON line in all, from rank 0, and both
+    ranks exit 0."""
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), "bench.py", "--impl", "reference",
+           "--gpus", "2", "--steps", "1", "--warmup", "3", "--ref-total-s", "2"]
+    r = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip().startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2
 
 
 def test_fewer_than_three_warmup_steps_are_rejected():
