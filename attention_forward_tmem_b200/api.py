@@ -8,6 +8,8 @@ Mirrors the pages' API surface:
   * :func:`attn_fwd` -- the attention forward of "Core 注意力" (section
     "选择最窄的入口", PyTorch SDPA contract with GQA) and of "MLA Prefill"
     (packed layout, qSeqLen/kvSeqLen, QRope/kRope, headNum/kvHeadNum/qkScale).
+  * :func:`scaled_dot_product_attention` -- the same forward under the
+    PyTorch SDPA signature itself, for callers of that entry.
   * :class:`BlockKVCache` -- the rolling cache of "Core 注意力", section
     "Block KV cache 的调用顺序" (before_update -> update -> cached_k/cached_v
     -> after_update).
@@ -158,6 +160,64 @@ def attn_fwd(q, k, v, *, qrope=None, krope=None, q_seqlen=None, kv_seqlen=None, 
                                  float(qk_scale), int(mask_type), ctypes.byref(od), _stream(stream))
     _check(st)
     return (out, lse) if want_lse else out
+
+
+def scaled_dot_product_attention(query, key, value, attn_mask=None, dropout_p=0.0, is_causal=False,
+                                 scale=None, enable_gqa=False, *, out=None, stream=None):
+    """The ``torch.nn.functional.scaled_dot_product_attention`` contract that
+    "Core 注意力" (section "选择最窄的入口") gives its entry, for inference,
+    on this library's kernels (argument mapping onto :func:`attn_fwd`).
+
+    ``query`` [B, Hq, L, E] or [Hq, L, E]; ``key`` / ``value`` [B, Hkv, S, E]
+    / [B, Hkv, S, Ev] (same rank as ``query``).  ``attn_mask``: bool (True =
+    the key takes part) or float (added to the scaled scores), broadcastable
+    to [B, Hq, L, S].  ``is_causal``: query i sees keys j <= i, aligned at the
+    top-left as in torch; with L == S that is the library's causal mask,
+    otherwise an explicit keep-mask is passed.  ``scale`` defaults to
+    1/sqrt(E).  ``enable_gqa``: Hq may be a multiple of Hkv (consecutive query
+    heads share a key head).  ``dropout_p`` must be 0.
+
+    One difference from torch: a row whose keys are all masked gives zeros
+    (torch gives NaN).
+    """
+    if dropout_p != 0.0:
+        raise ValueError("dropout_p must be 0: this is the inference forward")
+    if is_causal and attn_mask is not None:
+        raise ValueError("attn_mask and is_causal cannot both be given (as in torch)")
+    squeeze = query.dim() == 3
+    if squeeze:
+        query, key, value = query.unsqueeze(0), key.unsqueeze(0), value.unsqueeze(0)
+    if query.dim() != 4 or key.dim() != 4 or value.dim() != 4:
+        raise ValueError("query / key / value must all be [B, H, L, E] or all [H, L, E]")
+    hq, hk = query.shape[1], key.shape[1]
+    if hq != hk and not enable_gqa:
+        raise ValueError(f"{hq} query heads against {hk} key heads needs enable_gqa=True (as in torch)")
+    lq, lk = query.shape[2], key.shape[2]
+    mask, mask_type = None, MaskType.NONE
+    if is_causal:
+        if lq == lk:
+            mask_type = MaskType.CAUSAL
+        else:
+            mask = torch.ones(lq, lk, dtype=torch.bool, device=query.device).tril()
+            mask_type = MaskType.BOOL_KEEP
+    elif attn_mask is not None:
+        mask = attn_mask
+        if mask.dtype == torch.bool:
+            mask_type = MaskType.BOOL_KEEP
+        else:
+            if mask.dtype not in (torch.float32, query.dtype):
+                mask = mask.float()
+            mask_type = MaskType.ADDITIVE
+    if mask is not None:
+        if mask.dim() > 4:
+            raise ValueError("attn_mask must be broadcastable to [B, H, L, S]")
+        while mask.dim() < 4:
+            mask = mask.unsqueeze(0)
+    if out is not None and squeeze:
+        out = out.unsqueeze(0)
+    res = attn_fwd(query, key, value, mask=mask, mask_type=mask_type, qk_scale=scale, out=out,
+                   stream=stream)
+    return res.squeeze(0) if squeeze else res
 
 
 def merge(out_parts, lse_parts, *, out=None, lse=None, stream=None):
