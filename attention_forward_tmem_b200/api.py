@@ -163,7 +163,7 @@ def attn_fwd(q, k, v, *, qrope=None, krope=None, q_seqlen=None, kv_seqlen=None, 
 
 
 def scaled_dot_product_attention(query, key, value, attn_mask=None, dropout_p=0.0, is_causal=False,
-                                 scale=None, enable_gqa=False, *, out=None, stream=None):
+                                 scale=None, enable_gqa=False, *, backend=None, out=None, stream=None):
     """The ``torch.nn.functional.scaled_dot_product_attention`` contract that
     "Core 注意力" (section "选择最窄的入口") gives its entry, for inference,
     on this library's kernels (argument mapping onto :func:`attn_fwd`).
@@ -175,7 +175,10 @@ def scaled_dot_product_attention(query, key, value, attn_mask=None, dropout_p=0.
     top-left as in torch; with L == S that is the library's causal mask,
     otherwise an explicit keep-mask is passed.  ``scale`` defaults to
     1/sqrt(E).  ``enable_gqa``: Hq may be a multiple of Hkv (consecutive query
-    heads share a key head).  ``dropout_p`` must be 0.
+    heads share a key head).  ``dropout_p`` must be 0.  ``backend`` is
+    accepted for call compatibility with the page's entry, which selects a
+    provider with it; this library has one provider, its sm_100a kernels,
+    whatever is named.
 
     One difference from torch: a row whose keys are all masked gives zeros
     (torch gives NaN).
@@ -280,9 +283,25 @@ class BlockKVCache:
     CUDA device.  ``sink_size + window_size == L``; both multiples of
     ``chunk_size``.  State transitions are checked by the library; a call out
     of order raises :class:`WfError` with status ``WF_ERR_ORDER``.
+
+    The constructor form of "Core 注意力" ("Block KV cache 的调用顺序") is
+    accepted too: ``BlockKVCache(k_shape=..., v_shape=..., seq_dim=...,
+    chunk_size=..., window_size=..., device=..., dtype=...)`` allocates zeroed
+    buffers (``device`` must be a CUDA device).
     """
 
-    def __init__(self, k_buf, v_buf, *, seq_dim=2, chunk_size, window_size, sink_size=0):
+    def __init__(self, k_buf=None, v_buf=None, *, seq_dim=2, chunk_size, window_size, sink_size=0,
+                 k_shape=None, v_shape=None, device="cuda", dtype=torch.bfloat16):
+        bufs = (k_buf is not None, v_buf is not None)
+        shapes = (k_shape is not None, v_shape is not None)
+        if not ((all(bufs) and not any(shapes)) or (all(shapes) and not any(bufs))):
+            raise ValueError("give either k_buf and v_buf, or k_shape and v_shape")
+        if all(shapes):
+            if torch.device(device).type != "cuda":
+                raise WfError(L.WF_ERR_INVALID_ARG,
+                              "tensors must be on a CUDA device (this library has no CPU path)")
+            k_buf = torch.zeros(k_shape, dtype=dtype, device=device)
+            v_buf = torch.zeros(v_shape, dtype=dtype, device=device)
         _require_cuda(k_buf, v_buf)
         self.k_buf, self.v_buf = k_buf, v_buf
         self.seq_dim = seq_dim
@@ -296,10 +315,8 @@ class BlockKVCache:
     def allocate(cls, k_shape, v_shape, *, seq_dim=2, chunk_size, window_size, sink_size=0,
                  device="cuda", dtype=torch.bfloat16):
         """Allocate zeroed buffers of the given shapes and wrap them."""
-        kb = torch.zeros(k_shape, dtype=dtype, device=device)
-        vb = torch.zeros(v_shape, dtype=dtype, device=device)
-        return cls(kb, vb, seq_dim=seq_dim, chunk_size=chunk_size, window_size=window_size,
-                   sink_size=sink_size)
+        return cls(k_shape=k_shape, v_shape=v_shape, seq_dim=seq_dim, chunk_size=chunk_size,
+                   window_size=window_size, sink_size=sink_size, device=device, dtype=dtype)
 
     def __del__(self):
         h = getattr(self, "_h", None)

@@ -94,3 +94,27 @@ def test_three_dim_inputs(captured):
     (qq, kk, vv, kw), = captured
     assert qq.shape == (1, 4, 16, 8) and vv.shape == (1, 4, 16, 6)
     assert out.shape == (4, 16, 6)
+
+
+def test_backend_keyword_is_accepted(captured):
+    q, k, v = _qkv()
+    api.scaled_dot_product_attention(q, k, v, dropout_p=0.0, backend="math")
+    (_, _, _, kw), = captured
+    assert kw["mask_type"] == api.MaskType.NONE
+
+
+def test_cache_constructor_forms():
+    """The page's keyword form (shapes, device, dtype) and the buffer form;
+    anything mixed is refused, and a host device is refused loudly."""
+    shape = (1, 1, 4, 2)
+    with pytest.raises(ValueError, match="either"):
+        api.BlockKVCache(chunk_size=2, window_size=4)
+    with pytest.raises(ValueError, match="either"):
+        api.BlockKVCache(torch.zeros(shape), k_shape=shape, v_shape=shape, chunk_size=2, window_size=4)
+    with pytest.raises(ValueError, match="either"):
+        api.BlockKVCache(k_shape=shape, chunk_size=2, window_size=4)
+    with pytest.raises(api.WfError, match="no CPU path"):
+        api.BlockKVCache(k_shape=shape, v_shape=(1, 1, 4, 3), seq_dim=2, chunk_size=2, window_size=4,
+                         device="cpu", dtype=torch.float32)
+    with pytest.raises(api.WfError, match="no CPU path"):
+        api.BlockKVCache(torch.zeros(shape), torch.zeros(1, 1, 4, 3), chunk_size=2, window_size=4)
