@@ -7,7 +7,8 @@ library is missing or no sm_100 device is present, the calls raise.
 
 Importing the package does not load the library; the first API call does.
 """
-__all__ = ["attn_fwd", "BlockKVCache", "device_status", "MaskType", "WfError"]
+__all__ = ["attn_fwd", "scaled_dot_product_attention", "merge", "dca", "BlockKVCache", "device_status",
+           "MaskType", "WfError"]
 
 
 def __getattr__(name):
