@@ -27,7 +27,7 @@ STATUS_NAMES = {0: "WF_OK", 1: "WF_ERR_INVALID_ARG", 2: "WF_ERR_UNSUPPORTED", 3:
 WF_F32, WF_BF16, WF_F16, WF_U8, WF_I32 = 0, 1, 2, 3, 4
 
 # wf_mask_type_t
-WF_MASK_NONE, WF_MASK_CAUSAL, WF_MASK_BOOL_KEEP, WF_MASK_ADDITIVE = 0, 1, 2, 3
+WF_MASK_NONE, WF_MASK_CAUSAL, WF_MASK_BOOL_KEEP, WF_MASK_ADDITIVE, WF_MASK_CAUSAL_TOP_LEFT = 0, 1, 2, 3, 4
 
 
 class WfTensor(ctypes.Structure):
@@ -59,6 +59,7 @@ SIGNATURES = {
     "wf_kvcache_get_state": (_I32, [_P, ctypes.POINTER(_I64), ctypes.POINTER(_I64),
                                     ctypes.POINTER(_I64), ctypes.POINTER(_I64),
                                     ctypes.POINTER(_I32)]),
+    "wf_kvcache_set_state": (_I32, [_P, _I64]),
     "wf_kvcache_gather_logical": (_I32, [_P, _T, _T, _P]),
     "wf_kvcache_destroy": (None, [_P]),
     "wf_get_device_status": (_I32, [_P]),

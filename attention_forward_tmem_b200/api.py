@@ -36,6 +36,7 @@ class MaskType(enum.IntEnum):
     CAUSAL = L.WF_MASK_CAUSAL
     BOOL_KEEP = L.WF_MASK_BOOL_KEEP
     ADDITIVE = L.WF_MASK_ADDITIVE
+    CAUSAL_TOP_LEFT = L.WF_MASK_CAUSAL_TOP_LEFT
 
 
 _DTYPES = {torch.float32: L.WF_F32, torch.bfloat16: L.WF_BF16, torch.float16: L.WF_F16,
@@ -198,11 +199,9 @@ def scaled_dot_product_attention(query, key, value, attn_mask=None, dropout_p=0.
     lq, lk = query.shape[2], key.shape[2]
     mask, mask_type = None, MaskType.NONE
     if is_causal:
-        if lq == lk:
-            mask_type = MaskType.CAUSAL
-        else:
-            mask = torch.ones(lq, lk, dtype=torch.bool, device=query.device).tril()
-            mask_type = MaskType.BOOL_KEEP
+        # torch's is_causal is top-left aligned (key j visible to query i iff
+        # j <= i); the kernel generates it, as it does the bottom-right form
+        mask_type = MaskType.CAUSAL if lq == lk else MaskType.CAUSAL_TOP_LEFT
     elif attn_mask is not None:
         mask = attn_mask
         if mask.dtype == torch.bool:
@@ -379,6 +378,11 @@ class BlockKVCache:
                                              ctypes.byref(slot), ctypes.byref(vis),
                                              ctypes.byref(ph)))
         return cur.value, com.value, slot.value, vis.value, ph.value
+
+    def set_state(self, committed_idx: int) -> None:
+        """Resume at chunk ``committed_idx`` (-1: none) as the last committed
+        chunk, for buffers restored by the caller (``wf_kvcache_set_state``)."""
+        _check(L.load().wf_kvcache_set_state(self._h, int(committed_idx)))
 
     def gather_logical(self, stream=None):
         """Copy of the visible tokens in logical chunk order (buffer layout)."""

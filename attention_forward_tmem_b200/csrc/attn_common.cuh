@@ -85,7 +85,7 @@ __device__ __forceinline__ TileInfo tile_info(const AttnParams &p, int32_t t, in
   const int32_t u0 = u * p.unit_rows;
   ti.q0 = u0 + sub * kBlockM;
   ti.qrow = (p.varlen ? __ldg(p.ws + p.sl.cu_q + ti.b) : 0) + ti.q0;
-  ti.off = ti.lk - ti.lq;
+  ti.off = p.causal_top_left ? 0 : ti.lk - ti.lq;   // causal: last visible key of row i is i + off
   int32_t kend = ti.q0 < ti.lq ? ti.lk : 0;            // no valid row: nothing to do
   if (causal) {
     const int32_t last = min(ti.q0 + kBlockM, ti.lq);   // one past the last valid row

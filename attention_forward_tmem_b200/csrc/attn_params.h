@@ -54,6 +54,7 @@ struct alignas(64) AttnParams {
   const void *mask;
   int64_t m_sb, m_sh, m_si, m_sj;                // element strides of the mask (0 = broadcast)
   int32_t mask_kind, mask_dtype;
+  int32_t causal_top_left;                      // causal: key j visible to row i iff j <= i
   int32_t batch, hq, hkv, group;
   int32_t lq, lk;                                // dense lengths
   int32_t varlen;

@@ -324,6 +324,17 @@ wf_status_t wf_kvcache_get_state(const wf_kvcache_t *c, int64_t *cur, int64_t *c
   return WF_OK;
 }
 
+wf_status_t wf_kvcache_set_state(wf_kvcache_t *c, int64_t committed) {
+  clear_error();
+  if (!c) return fail(WF_ERR_INVALID_ARG, "cache is NULL");
+  if (c->phase != kIdle)
+    return fail(WF_ERR_ORDER, "set_state while chunk %lld is in progress", (long long)c->current);
+  if (committed < -1) return fail(WF_ERR_INVALID_ARG, "committed index %lld < -1", (long long)committed);
+  c->committed = committed;
+  c->current = committed;
+  return WF_OK;
+}
+
 wf_status_t wf_kvcache_gather_logical(wf_kvcache_t *c, wf_tensor_t *k_out, wf_tensor_t *v_out, void *stream) {
   clear_error();
   wf_status_t st;

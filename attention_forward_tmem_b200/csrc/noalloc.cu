@@ -56,6 +56,13 @@ wf_status_t schedule_array(int dev, int32_t **out, int32_t **counters) {
 
 }  // namespace
 
+// Forget the looked-up addresses (wf_shutdown): after a device reset the
+// next call looks them up again.
+void forget_noalloc_addresses() {
+  std::lock_guard<std::mutex> lock(g_mu);
+  for (int i = 0; i < 64; ++i) g_sched_ptr[i] = g_counter_ptr[i] = nullptr;
+}
+
 cudaError_t reset_noalloc_counters() {
   const int32_t zero[4] = {0, 0, 0, 0};
   return cudaMemcpyToSymbol(g_noalloc_counters, zero, sizeof(zero));
@@ -75,8 +82,8 @@ extern "C" wf_status_t wf_attn_fwd_varlen_noalloc(
     return fail(WF_ERR_INVALID_ARG, "q, k, v, qSeqLen, kvSeqLen and out are required");
   if (q->dtype != WF_BF16)
     return fail(WF_ERR_UNSUPPORTED, "the allocation-free entry point takes bf16 tensors only");
-  if (maskType != WF_MASK_NONE && maskType != WF_MASK_CAUSAL)
-    return fail(WF_ERR_UNSUPPORTED, "packed sequences take maskType NONE or CAUSAL");
+  if (maskType != WF_MASK_NONE && maskType != WF_MASK_CAUSAL && maskType != WF_MASK_CAUSAL_TOP_LEFT)
+    return fail(WF_ERR_UNSUPPORTED, "packed sequences take maskType NONE, CAUSAL or CAUSAL_TOP_LEFT");
   if (!std::isfinite(qkScale)) return fail(WF_ERR_INVALID_ARG, "qkScale is not finite");
   if ((qRope == nullptr) != (kRope == nullptr))
     return fail(WF_ERR_INVALID_ARG, "qRope and kRope are given together or not at all");
@@ -171,7 +178,8 @@ extern "C" wf_status_t wf_attn_fwd_varlen_noalloc(
   p.o_sb = 0;
   p.o_sh = out->stride[1];
   p.o_si = out->stride[0];
-  p.mask_kind = maskType;
+  p.mask_kind = maskType == WF_MASK_CAUSAL_TOP_LEFT ? kMaskCausal : maskType;
+  p.causal_top_left = maskType == WF_MASK_CAUSAL_TOP_LEFT ? 1 : 0;
   p.batch = (int32_t)B;
   p.hq = headNum;
   p.hkv = kvHeadNum;

@@ -366,7 +366,7 @@ static wf_status_t attn_fwd_impl(const wf_tensor_t *q, const wf_tensor_t *qRope,
   const int32_t dt = q->dtype;
   if (dt != WF_BF16 && dt != WF_F16 && dt != WF_F32)
     return fail(WF_ERR_UNSUPPORTED, "q dtype %d: only WF_BF16, WF_F16 and WF_F32 are implemented", dt);
-  if (maskType < WF_MASK_NONE || maskType > WF_MASK_ADDITIVE)
+  if (maskType < WF_MASK_NONE || maskType > WF_MASK_CAUSAL_TOP_LEFT)
     return fail(WF_ERR_INVALID_ARG, "maskType %d out of range", maskType);
   if (!std::isfinite(qkScale)) return fail(WF_ERR_INVALID_ARG, "qkScale is not finite");
   if ((qSeqLen == nullptr) != (kvSeqLen == nullptr))
@@ -581,7 +581,8 @@ static wf_status_t attn_fwd_impl(const wf_tensor_t *q, const wf_tensor_t *qRope,
   p.m_sh = ms[1];
   p.m_si = ms[2];
   p.m_sj = ms[3];
-  p.mask_kind = maskType;
+  p.mask_kind = maskType == WF_MASK_CAUSAL_TOP_LEFT ? kMaskCausal : maskType;
+  p.causal_top_left = maskType == WF_MASK_CAUSAL_TOP_LEFT ? 1 : 0;
   p.mask_dtype = mask_dtype;
   p.batch = (int32_t)d.batch;
   p.hq = headNum;
@@ -771,7 +772,11 @@ void wf_shutdown(void) {
     }
   }
   g_scratch.clear();
+  // cached device addresses (status word, fixed arrays): looked up again on
+  // next use, so that calls after a device reset see the new addresses
+  g_devices.clear();
   cudaSetDevice(cur);
+  forget_noalloc_addresses();
 }
 
 }  // extern "C"

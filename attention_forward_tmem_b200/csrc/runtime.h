@@ -53,6 +53,8 @@ cudaError_t launch_fill_f32(float *dst, int64_t n, float v, cudaStream_t stream)
 // Zero the allocation-free entry's work-item counters on the current device
 // (noalloc.cu); used after a launch was aborted.
 cudaError_t reset_noalloc_counters();
+// Forget the fixed arrays' device addresses (looked up again on next use).
+void forget_noalloc_addresses();
 // 4-d TMA map (D, rows, heads, batch), (128 bytes of D) x 128 rows box,
 // 128-byte swizzle, zero fill outside the tensor; strides in elements.
 wf_status_t make_map(CUtensorMap *map, const void *base, int32_t dtype, int64_t d, int64_t rows,

@@ -71,12 +71,18 @@ typedef enum wf_dtype {
 /* maskType.  [P2] table row "maskType" (UNDEFINED / SPEC / MASK_FREE) and row
  * "Mask" (CAUSAL_MASK may pass nullptr); [P1] example section for the two
  * explicit mask kinds.  ATB names map as: UNDEFINED -> NONE; CAUSAL_MASK,
- * MASK_FREE, SPEC -> CAUSAL (generated in the kernel; no mask tensor read). */
+ * MASK_FREE, SPEC -> CAUSAL (generated in the kernel; no mask tensor read).
+ * Both causal kinds are bottom-right or top-left alignments of the same
+ * predicate; rows that see no key give 0 (and LSE -inf). */
 typedef enum wf_mask_type {
     WF_MASK_NONE = 0,
     WF_MASK_CAUSAL = 1,     /* key j visible to query i iff j <= i + (Lk - Lq) */
     WF_MASK_BOOL_KEEP = 2,  /* mask dtype WF_U8, nonzero = keep               */
-    WF_MASK_ADDITIVE = 3    /* mask dtype = q dtype or WF_F32, added to scores */
+    WF_MASK_ADDITIVE = 3,   /* mask dtype = q dtype or WF_F32, added to scores */
+    WF_MASK_CAUSAL_TOP_LEFT = 4  /* key j visible to query i iff j <= i: the
+                                  * alignment of PyTorch SDPA's is_causal ([P1]
+                                  * "选择最窄的入口"); the same as WF_MASK_CAUSAL
+                                  * when Lq == Lk.  Generated in the kernel. */
 } wf_mask_type_t;
 
 /* Tensor descriptor: up to 4 dims, strides in elements, caller-owned data. */
@@ -256,17 +262,24 @@ wf_status_t wf_attn_fwd_debug(const wf_tensor_t *q, const wf_tensor_t *qRope,
  * captured into CUDA graphs that must leave the allocator alone, runtimes
  * that give the whole device to a pool at start-up, fixed memory budgets).
  *
- * Arguments as in wf_attn_fwd's packed layout (no mask; maskType NONE or
- * CAUSAL; all tensors WF_BF16).  Instead of an allocated workspace, the
- * schedule tables live in a fixed array inside the library: 65536 int32
- * words (256 KiB) on every GPU that loads the library, held until the
- * process exits.  A call needs 4 * batch + 5 words (batch <= 16382); larger
- * calls return WF_ERR_INVALID_ARG and launch nothing.  The first call on a device looks the array's address up
- * (cudaGetSymbolAddress); make that first call before any stream capture.
- * All calls share the array: calls whose work overlaps on the GPU (e.g. on
- * different streams) race; calls in order on one stream do not, as each
- * rewrites every word it reads.  Other dtypes and the dense layout return
- * WF_ERR_UNSUPPORTED (the dense bf16 path of wf_attn_fwd allocates nothing).
+ * Arguments as in wf_attn_fwd's packed layout (no mask; maskType NONE,
+ * CAUSAL or CAUSAL_TOP_LEFT; all tensors WF_BF16).  Instead of an allocated
+ * workspace, the schedule tables live in a fixed array inside the library:
+ * 65536 int32 words (256 KiB) on every GPU that loads the library, held until
+ * the process exits; the work-item counters live in a fixed 4-word array.  A
+ * call needs 4 * batch + 5 words (batch <= 16382); larger calls return
+ * WF_ERR_INVALID_ARG and launch nothing.  The first call on a device looks
+ * the arrays' addresses up (cudaGetSymbolAddress); make that first call
+ * before any stream capture.  The addresses are kept for the life of the
+ * process: after a cudaDeviceReset, call wf_shutdown (which forgets them)
+ * before calling again.  All calls share the arrays: calls whose work
+ * overlaps on the GPU (e.g. on different streams) race; calls in order on
+ * one stream do not, as each rewrites every word it reads.  Other dtypes and
+ * the explicit mask kinds return WF_ERR_UNSUPPORTED, tensors that are not
+ * 3-d (the dense layout) WF_ERR_INVALID_ARG; split-KV and the LSE output are
+ * not offered here.  wf_attn_fwd itself is
+ * no substitute for such callers in any layout: its first call on each
+ * (device, stream) allocates a workspace of at least 1 MiB with cudaMalloc.
  */
 wf_status_t wf_attn_fwd_varlen_noalloc(const wf_tensor_t *q, const wf_tensor_t *qRope,
                                        const wf_tensor_t *k, const wf_tensor_t *kRope,
@@ -369,6 +382,16 @@ wf_status_t wf_kvcache_get_state(const wf_kvcache_t *cache, int64_t *cur_idx,
                                  int64_t *committed_idx, int64_t *write_slot,
                                  int64_t *visible_len, int32_t *phase);
 
+/* Restore the rolling state: chunk `committed_idx` (-1: none) becomes the
+ * last committed chunk, with no chunk in progress, as if the calls up to
+ * after_update(committed_idx) had run on this handle.  For resuming a cache
+ * whose buffers the caller has restored (e.g. from a checkpoint); the buffers
+ * are not touched, and holding the matching contents is the caller's part.
+ * Host only.  WF_ERR_ORDER while a chunk is in progress (state unchanged),
+ * WF_ERR_INVALID_ARG for committed_idx < -1.  The pages have no counterpart
+ * (their cache lives in one process from chunk 0 on). */
+wf_status_t wf_kvcache_set_state(wf_kvcache_t *cache, int64_t committed_idx);
+
 /* Copy the visible tokens in LOGICAL chunk order (sink chunks, then the
  * window's chunks oldest first) into k_out / v_out, [B, H, vis, D] (or the
  * seq_dim = 1 form).  Allowed in the same phases as wf_kvcache_cached. */
@@ -397,7 +420,10 @@ const char *wf_last_error_message(void);
 /* Library version (WF_ATTN_VERSION). */
 int32_t wf_version(void);
 
-/* Free the per-device workspaces.  Call with no work in flight. */
+/* Free the per-device workspaces and forget the cached device addresses (the
+ * status word, the fixed arrays of wf_attn_fwd_varlen_noalloc); the next call
+ * sets them up again.  Call with no work in flight, and after a
+ * cudaDeviceReset before any other call of the library. */
 void wf_shutdown(void);
 
 #ifdef __cplusplus

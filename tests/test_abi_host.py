@@ -338,6 +338,31 @@ def test_cache_order_errors_on_host(lib):
     lib.wf_kvcache_destroy(h)
 
 
+def test_cache_set_state_resumes_the_rolling_order(lib):
+    """set_state(c) leaves the handle as after_update(c): the next legal
+    chunk indices are c (overwrite) and c + 1, the write slot and visible
+    length follow the ring; refused while a chunk is in progress."""
+    st, h = _cache(lib)                    # L 8, chunk 2, sink 2, window 6: 4 slots
+    assert st == L.WF_OK
+    assert lib.wf_kvcache_set_state(h, -2) == L.WF_ERR_INVALID_ARG
+    assert lib.wf_kvcache_set_state(h, 5) == L.WF_OK
+    assert _state(lib, h) == (5, 5, 1 + (5 - 1) % 3, 8, 0)
+    assert lib.wf_kvcache_before_update(h, 7) == L.WF_ERR_ORDER
+    assert lib.wf_kvcache_before_update(h, 6) == L.WF_OK
+    assert _state(lib, h) == (6, 5, 1 + (6 - 1) % 3, 8, 1)
+    assert lib.wf_kvcache_set_state(h, 2) == L.WF_ERR_ORDER          # chunk 6 in progress
+    assert _state(lib, h) == (6, 5, 1 + (6 - 1) % 3, 8, 1)
+    lib.wf_kvcache_destroy(h)
+    st, h = _cache(lib)
+    assert lib.wf_kvcache_set_state(h, 0) == L.WF_OK
+    assert _state(lib, h) == (0, 0, 0, 2, 0)
+    assert lib.wf_kvcache_set_state(h, -1) == L.WF_OK                # back to the empty cache
+    assert _state(lib, h) == (-1, -1, -1, 0, 0)
+    assert lib.wf_kvcache_before_update(h, 1) == L.WF_ERR_ORDER
+    assert lib.wf_kvcache_before_update(h, 0) == L.WF_OK
+    lib.wf_kvcache_destroy(h)
+
+
 def _state(lib, h):
     cur, com, slot, vis = (ctypes.c_int64() for _ in range(4))
     ph = ctypes.c_int32()

@@ -1,8 +1,8 @@
 """api.scaled_dot_product_attention: the PyTorch SDPA signature of "Core 注意力"
 (section "选择最窄的入口") mapped onto attn_fwd.  Host-side checks of the
-mapping (the call into the library is captured), and of the one piece of
-semantics the mapping builds itself, the top-left causal mask for L != S,
-against torch's own is_causal on the CPU."""
+mapping (the call into the library is captured), and of the predicate of
+the top-left causal kind that is_causal maps to when L != S, against torch's
+own is_causal on the CPU."""
 import math
 
 import pytest
@@ -58,15 +58,18 @@ def test_plain_gqa_scale_and_causal_square(captured):
 
 @pytest.mark.parametrize("L,S", [(5, 12), (12, 5)])
 def test_causal_with_unequal_lengths_is_top_left(captured, L, S):
+    """is_causal with L != S maps to the kernel's top-left causal kind (no
+    mask tensor); its documented predicate, key j visible to query i iff
+    j <= i, reproduces torch's own is_causal."""
     q, k, v = _qkv(L=L, S=S)
     api.scaled_dot_product_attention(q, k, v, is_causal=True)
     (_, _, _, kw), = captured
-    assert kw["mask_type"] == api.MaskType.BOOL_KEEP
-    m = kw["mask"]
-    assert m.shape == (1, 1, L, S) and m.dtype == torch.bool
-    # the keep-mask reproduces torch's own is_causal, which is top-left aligned
+    assert kw["mask_type"] == api.MaskType.CAUSAL_TOP_LEFT and kw["mask"] is None
+    i = torch.arange(L)[:, None]
+    j = torch.arange(S)[None, :]
+    keep = j <= i
     want = F.scaled_dot_product_attention(q, k, v, is_causal=True)
-    got = F.scaled_dot_product_attention(q, k, v, attn_mask=m)
+    got = F.scaled_dot_product_attention(q, k, v, attn_mask=keep)
     finite = torch.isfinite(want).all(-1)             # torch gives NaN rows where no key is visible
     assert torch.allclose(got[finite], want[finite], atol=1e-12)
 
