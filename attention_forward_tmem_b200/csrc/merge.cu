@@ -11,7 +11,9 @@
 // exponentiating.
 //
 // One warp per row, four consecutive columns per lane per pass (128 columns
-// a pass); HBM-bound: it reads S partial rows and writes one.
+// a pass); HBM-bound: it reads S partial rows and writes one.  With at most
+// four parts (the split-KV case) every load of a row (the parts' LSEs and
+// their columns) is issued at once, so a row costs one memory latency.
 #include <algorithm>
 #include <cstdint>
 #include <cuda_bf16.h>
@@ -129,6 +131,54 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(const __grid_co
     mp.lse[i0 * mp.e_s0 + i1 * mp.e_s1 + i2 * mp.e_s2] = empty ? -INFINITY : top + __log2f(total) * kLn2M;
 }
 
+// At most kFewParts parts and Dv <= 128: each lane loads every part's LSE
+// (the same words in every lane) and its four columns of every part in one
+// batch, then combines them without shuffles.
+constexpr int kFewParts = 4;
+__global__ void __launch_bounds__(kMergeWarps * 32) merge_few_kernel(const __grid_constant__ MergeParams mp) {
+  pdl_wait();
+  pdl_trigger();
+  int64_t rows = mp.rows;
+  if (mp.sched) {
+    if (mp.sched[1] != 0) return;
+    rows = min(rows, (int64_t)mp.sched[mp.sched_tokens] * mp.n2);
+  }
+  const int64_t r = (int64_t)blockIdx.x * kMergeWarps + (threadIdx.x >> 5);
+  if (r >= rows) return;
+  const int lane = threadIdx.x & 31;
+  const int c = lane * 4;
+  const bool col = c < mp.dv;
+  float ls[kFewParts], v[kFewParts][4];
+#pragma unroll
+  for (int s = 0; s < kFewParts; ++s) {
+    ls[s] = s < mp.n_split ? mp.lses[s * mp.l_ss + r * mp.l_sr] : -INFINITY;
+    v[s][0] = v[s][1] = v[s][2] = v[s][3] = 0.f;
+    if (s < mp.n_split && col) load4(mp.parts, s * mp.p_ss + r * mp.p_sr + c, mp.parts_type, v[s]);
+  }
+  float top = ls[0];
+#pragma unroll
+  for (int s = 1; s < kFewParts; ++s) top = fmaxf(top, ls[s]);
+  const bool empty = top == -INFINITY;
+  float w[kFewParts], total = 0.f;
+#pragma unroll
+  for (int s = 0; s < kFewParts; ++s) {
+    w[s] = (empty || ls[s] == -INFINITY) ? 0.f : ex2_approx((ls[s] - top) * kLog2eM);
+    total += w[s];
+  }
+  const float inv = empty ? 0.f : 1.f / total;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int s = 0; s < kFewParts; ++s)
+    if (w[s] != 0.f)                                  // weight 0: its row may be anything
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[e] = fmaf(w[s] * inv, v[s][e], acc[e]);
+  const int64_t i2 = r % mp.n2, i01 = r / mp.n2;
+  const int64_t i1 = i01 % mp.n1, i0 = i01 / mp.n1;
+  if (col) store4(mp.out, i0 * mp.o_s0 + i1 * mp.o_s1 + i2 * mp.o_s2 + c, mp.out_type, acc);
+  if (mp.lse && lane == 0)
+    mp.lse[i0 * mp.e_s0 + i1 * mp.e_s1 + i2 * mp.e_s2] = empty ? -INFINITY : top + __log2f(total) * kLn2M;
+}
+
 __global__ void fill_f32_kernel(float *dst, int64_t n, float v) {
   pdl_wait();
   pdl_trigger();
@@ -148,6 +198,9 @@ cudaError_t launch_merge(const MergeParams &mp, cudaStream_t stream) {
   if (mp.rows <= 0) return cudaSuccess;
   const int64_t blocks = (mp.rows + kMergeWarps - 1) / kMergeWarps;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  if (mp.n_split <= kFewParts && mp.dv <= 128)
+    return launch_pdl(merge_few_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kMergeWarps * 32), 0,
+                      stream, mp);
   return launch_pdl(merge_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kMergeWarps * 32), 0, stream, mp);
 }
 

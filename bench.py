@@ -35,6 +35,7 @@ for profilers).
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import math
@@ -183,12 +184,14 @@ def config_of(name):
 class Workload:
     """One step's inputs and the call that runs it through the public API."""
 
-    def __init__(self, name, device):
+    def __init__(self, name, device, seq_len=None):
         from attention_forward_tmem_b200 import api
         self.api = api
         self.name = name
         self.device = device
         w = W.WORKLOADS[name]
+        if seq_len and name in ("gqa_causal_prefill", "long_gqa_causal"):
+            w = dataclasses.replace(w, seq=seq_len)      # a shorter case of the same shape (profiling)
         self.w = w
         self.launches_per_step = 1
         if name in ("gqa_causal_prefill", "long_gqa_causal"):
@@ -206,6 +209,8 @@ class Workload:
         else:
             raise SystemExit(f"bench workload {name!r} is not a single-call workload")
         self.config = config_of(name)
+        if "seq_len" in self.config:
+            self.config["seq_len"] = w.seq
         self.out_host = None
 
     def to_device(self):
@@ -594,8 +599,8 @@ def reference_arm(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
-def make_workload(name, device):
-    return RollingWorkload(name, device) if name == "blockkv_rolling" else Workload(name, device)
+def make_workload(name, device, seq_len=None):
+    return RollingWorkload(name, device) if name == "blockkv_rolling" else Workload(name, device, seq_len)
 
 
 def measure(wl, timer, args):
@@ -710,6 +715,8 @@ def main():
                     help="reference arm: seconds of oracle work per step (0: from --ref-total-s)")
     ap.add_argument("--ref-total-s", type=float, default=150.0,
                     help="reference arm: target seconds for warm-up plus timed steps")
+    ap.add_argument("--seq-len", type=int, default=None,
+                    help="dense workloads: a shorter sequence of the same shape (profiling cases)")
     ap.add_argument("--no-extras", action="store_true",
                     help="time the headline workload only (no e2e, CPU baseline, other workloads or "
                          "comparison loop; for profilers)")
@@ -727,8 +734,9 @@ def main():
     timer = BlockTimer(args.steps, args.warmup, args.min_timed_s, dist_on)
     peaks, peak_kind = measured_peaks()
 
-    wl = make_workload(args.workload, device)
+    wl = make_workload(args.workload, device, args.seq_len)
     wl.to_device()
+    headline_config = dict(wl.config)
     ms, blocks, total_ms, clocks, extra = measure(wl, timer, args)
     ms = parallel.max_over_ranks(ms, device)
     value = wl.flops * world / (ms / 1e3) / 1e12
@@ -777,7 +785,7 @@ def main():
     if dist_on:
         torch.distributed.barrier()
     if rank == 0:
-        cfg = dict(config_of(args.workload))
+        cfg = headline_config
         cfg["parallelism"] = f"dp{world}" if world > 1 else "single GPU"
         cfg["l2"] = "inputs larger than L2 (no flush needed)"
         line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,

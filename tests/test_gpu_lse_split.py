@@ -220,17 +220,19 @@ def test_merge_of_gpu_halves_equals_full_attention():
 
 
 @pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
-def test_merge_against_oracle_merge(out_dtype):
-    """Parts from the oracle over three random disjoint key sets (fp32), some
+@pytest.mark.parametrize("n_sets", [3, 6])
+def test_merge_against_oracle_merge(out_dtype, n_sets):
+    """Parts from the oracle over random disjoint key sets (fp32; three sets
+    take the single-batch merge for few parts, six the general one), some
     rows with an empty set, one row empty everywhere; NaN planted in rows whose
     LSE is -inf must not leak."""
     g = torch.Generator().manual_seed(44)
     q = torch.randn(1, 3, 40, 64, generator=g)
     k = torch.randn(1, 3, 90, 64, generator=g)
     v = torch.randn(1, 3, 90, 96, generator=g)
-    owner = torch.randint(0, 3, (90,), generator=g)
+    owner = torch.randint(0, n_sets, (90,), generator=g)
     outs, lses = [], []
-    for s_ in range(3):
+    for s_ in range(n_sets):
         keep = (owner == s_).view(1, 1, 1, 90).expand(1, 3, 40, 90).clone()
         keep[:, :, 5] = False                    # row 5 empty everywhere
         if s_ == 1:
