@@ -184,12 +184,68 @@ __device__ __forceinline__ float softmax_row(const AttnParams &p, const TileInfo
       x[c] = (c <= lim) ? __uint_as_float(sr[c]) * p.scale_log2 : -INFINITY;
   } else {
     const int64_t mrow = (int64_t)ti.b * p.m_sb + (int64_t)ti.h * p.m_sh + (int64_t)row * p.m_si;
-    if (p.mask_kind == kMaskKeep) {
+    // A full tile of a mask whose keys are contiguous and 16-byte aligned is
+    // read with 16-byte loads: a thread's 128 entries in a few vector loads
+    // instead of 128 scattered element loads.
+    const int es = p.mask_kind == kMaskKeep ? 1 : (p.mask_dtype == kMaskF32 ? 4 : 2);
+    const uint8_t *mrow_k0 = reinterpret_cast<const uint8_t *>(p.mask) + (mrow + k0) * es;
+    const bool vec = p.m_sj == 1 && k0 + kBlockN <= ti.lk &&
+                     (reinterpret_cast<uintptr_t>(mrow_k0) & 15) == 0;
+    if (p.mask_kind == kMaskKeep && vec) {
+      uint32_t w[32];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint4 v = row_valid ? __ldg(reinterpret_cast<const uint4 *>(mrow_k0) + i) : make_uint4(0, 0, 0, 0);
+        w[4 * i] = v.x;
+        w[4 * i + 1] = v.y;
+        w[4 * i + 2] = v.z;
+        w[4 * i + 3] = v.w;
+      }
+#pragma unroll
+      for (int c = 0; c < 128; ++c) {
+        const bool keep = c <= lim && ((w[c >> 2] >> (8 * (c & 3))) & 0xffu) != 0u;
+        x[c] = keep ? __uint_as_float(sr[c]) * p.scale_log2 : -INFINITY;
+      }
+    } else if (p.mask_kind == kMaskKeep) {
       const uint8_t *mp = reinterpret_cast<const uint8_t *>(p.mask) + mrow;
 #pragma unroll
       for (int c = 0; c < 128; ++c) {
         const bool keep = row_valid && c <= lim && mp[(int64_t)(k0 + c) * p.m_sj] != 0;
         x[c] = keep ? __uint_as_float(sr[c]) * p.scale_log2 : -INFINITY;
+      }
+    } else if (vec) {
+      // additive, 16 entries at a time (one or two 16-byte loads per 8)
+#pragma unroll
+      for (int c0 = 0; c0 < 128; c0 += 16) {
+        float a[16];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint8_t *src = mrow_k0 + (int64_t)(c0 + 8 * h) * es;
+          if (p.mask_dtype == kMaskF32) {
+            const float4 u = row_valid ? __ldg(reinterpret_cast<const float4 *>(src)) : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 v = row_valid ? __ldg(reinterpret_cast<const float4 *>(src) + 1) : make_float4(0.f, 0.f, 0.f, 0.f);
+            a[8 * h + 0] = u.x; a[8 * h + 1] = u.y; a[8 * h + 2] = u.z; a[8 * h + 3] = u.w;
+            a[8 * h + 4] = v.x; a[8 * h + 5] = v.y; a[8 * h + 6] = v.z; a[8 * h + 7] = v.w;
+          } else {
+            const uint4 u = row_valid ? __ldg(reinterpret_cast<const uint4 *>(src)) : make_uint4(0, 0, 0, 0);
+            const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              float2 f;
+              if (p.mask_dtype == kMaskBF16)
+                f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&uw[i]));
+              else
+                f = __half22float2(*reinterpret_cast<const __half2 *>(&uw[i]));
+              a[8 * h + 2 * i] = f.x;
+              a[8 * h + 2 * i + 1] = f.y;
+            }
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const bool in = row_valid && c0 + c <= lim;
+          x[c0 + c] = in ? fmaf(a[c], kLog2e, __uint_as_float(sr[c0 + c]) * p.scale_log2) : -INFINITY;
+        }
       }
     } else {
 #pragma unroll

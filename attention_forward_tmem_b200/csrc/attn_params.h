@@ -1,6 +1,7 @@
 // attn_params.h -- kernel parameter block and launch table shared by the
 // attention kernels and the host runtime (internal; not part of the C ABI).
 #pragma once
+#include <atomic>
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -85,6 +86,25 @@ struct alignas(64) AttnParams {
 };
 
 using AttnLaunchFn = cudaError_t (*)(const AttnParams &, int grid, cudaStream_t);
+
+// Generation of the per-device settings (raised by wf_shutdown, after which a
+// device may have been reset): a kernel's shared-memory limit is set once per
+// device and generation instead of before every launch.
+extern std::atomic<uint32_t> g_setup_generation;
+
+template <typename K>
+cudaError_t ensure_smem_limit(K kern, int bytes) {
+  static std::atomic<uint32_t> done[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint32_t gen = g_setup_generation.load(std::memory_order_acquire);
+  std::atomic<uint32_t> *slot = dev >= 0 && dev < 64 ? &done[dev] : nullptr;
+  if (slot && slot->load(std::memory_order_acquire) == gen) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && slot) slot->store(gen, std::memory_order_release);
+  return e;
+}
 
 // Launch with programmatic stream serialization: the kernel may begin (its
 // prologue) while the previous launch on the stream finishes; every kernel of

@@ -54,6 +54,8 @@ size_t dtype_size(int32_t dtype) {
 
 // ----------------------------------------------------------- device state
 __device__ int32_t g_device_status;   // one status word per device
+// starts at 1 so that the zero-initialised per-kernel records read "not set"
+std::atomic<uint32_t> g_setup_generation{1};
 
 static std::mutex g_mu;
 static std::map<int, DeviceState> g_devices;
@@ -775,6 +777,7 @@ void wf_shutdown(void) {
   // cached device addresses (status word, fixed arrays): looked up again on
   // next use, so that calls after a device reset see the new addresses
   g_devices.clear();
+  g_setup_generation.fetch_add(1);
   cudaSetDevice(cur);
   forget_noalloc_addresses();
 }

@@ -648,7 +648,10 @@ def roofline_of(wl, ms, peaks, peak_kind):
 def page_example_latency(device, calls=200):
     """Latency of the page example (fp32, q [2,8,32,64], k [2,8,48,64],
     v [2,8,48,96]) without a mask, with its keep-mask and with its additive
-    mask: microseconds per call, back-to-back calls on one stream."""
+    mask, in microseconds per call: back-to-back calls through the public API
+    on one stream (CUDA events; the host's argument checks and launches set the
+    pace), the host time per call, and the device time per call (the same calls
+    captured in a CUDA graph and replayed)."""
     from attention_forward_tmem_b200 import api
     q, k, v, keep, add = (t.to(device) for t in W.page_example_masks())
     out = torch.empty(2, 8, 32, 96, device=device)
@@ -660,15 +663,38 @@ def page_example_latency(device, calls=200):
             fn()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0 = time.perf_counter()
         e0.record()
         for _ in range(calls):
             fn()
         e1.record()
+        t1 = time.perf_counter()
         torch.cuda.synchronize()
-        res[kind] = 1e3 * e0.elapsed_time(e1) / calls
+        per = 1e3 * e0.elapsed_time(e1) / calls
+        host = 1e6 * (t1 - t0) / calls
+        # device time alone: 20 calls in a graph, replayed
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for _ in range(20):
+                fn()
+        g.replay()
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(10):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        dev_us = 1e3 * e0.elapsed_time(e1) / 200
+        del g
+        res[kind] = {"us_per_call": per, "host_us_per_call": host, "device_us_per_call": dev_us}
     api.device_status()
-    res["note"] = ("us per call (V^T kernel + attention kernel, fp32 inputs / TF32 products), "
-                   f"{calls} back-to-back calls")
+    res["note"] = ("V^T kernel + attention kernel per call, fp32 inputs / TF32 products; "
+                   f"{calls} back-to-back calls; device time from a CUDA graph of 20 calls")
     return res
 
 

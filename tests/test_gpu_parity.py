@@ -160,6 +160,36 @@ def test_masks_bf16(kind, mdtype, bshape):
         assert torch.all(out[:, :, 5] == 0)
 
 
+@pytest.mark.parametrize("kind,mdtype,bshape", [
+    ("keep", torch.bool, "full"), ("keep", torch.bool, "keys_strided"),
+    ("add", torch.float32, "bcast"), ("add", torch.bfloat16, "full"),
+])
+def test_masks_full_aligned_tiles(kind, mdtype, bshape):
+    """Lk = 384 (three full key tiles, every mask row 16-byte aligned): the
+    16-byte vector loads of the mask; a mask whose key dim is strided takes the
+    element loads."""
+    B, Hq, Hk, Lq, Lk = 1, 4, 2, 200, 384
+    q, k, v = W.dense_inputs(B, Hq, Hk, Lq, Lk, 128, 128, torch.bfloat16, 14)
+    g = torch.Generator().manual_seed(15)
+    if kind == "keep":
+        if bshape == "keys_strided":
+            m = (torch.rand(1, 1, Lk, Lq, generator=g) < 0.7).transpose(2, 3)
+        else:
+            m = torch.rand(B, Hq, Lq, Lk, generator=g) < 0.7
+        m[..., 7, :] = False
+    else:
+        shp = (B, Hq, Lq, Lk) if bshape == "full" else (1, 1, Lq, Lk)
+        m = (torch.randn(*shp, generator=g) * 2).to(mdtype)
+        m[..., 3, 200:] = -math.inf
+    out = api.attn_fwd(q.to(DEV), k.to(DEV), v.to(DEV), mask=m.to(DEV), qk_scale=1 / math.sqrt(128))
+    api.device_status()
+    ref = oracle.sdpa(q, k, v, mask=m.float() if kind == "add" else m, mask_kind=kind,
+                      qk_scale=1 / math.sqrt(128))
+    compare(out, ref, torch.bfloat16, f"{kind} {mdtype} {bshape}")
+    if kind == "keep":
+        assert torch.all(out[:, :, 7] == 0)
+
+
 def test_output_guard_bands():
     """Writes stay inside `out`: canary rows before and after it are untouched."""
     B, Hq, Hk, L, D = 1, 2, 1, 200, 128
