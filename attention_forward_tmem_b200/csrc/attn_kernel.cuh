@@ -359,7 +359,8 @@ template <typename T, int DQK, int DROPE, int DV>
 cudaError_t launch_attn(const AttnParams &p, int grid, cudaStream_t stream) {
   using Cfg = AttnCfg<T, DQK, DROPE, DV>;
   auto kern = attn_fwd_kernel<T, DQK, DROPE, DV>;
-  cudaError_t e = ensure_smem_limit(kern, Cfg::kSmemBytes);
+  static SmemLimitRecord limit;       // this kernel's
+  cudaError_t e = limit.ensure(kern, Cfg::kSmemBytes);
   if (e != cudaSuccess) return e;
   return launch_pdl(kern, dim3(grid), dim3(kThreads), Cfg::kSmemBytes, stream, p);
 }

@@ -92,19 +92,22 @@ using AttnLaunchFn = cudaError_t (*)(const AttnParams &, int grid, cudaStream_t)
 // device and generation instead of before every launch.
 extern std::atomic<uint32_t> g_setup_generation;
 
-template <typename K>
-cudaError_t ensure_smem_limit(K kern, int bytes) {
-  static std::atomic<uint32_t> done[64];
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  const uint32_t gen = g_setup_generation.load(std::memory_order_acquire);
-  std::atomic<uint32_t> *slot = dev >= 0 && dev < 64 ? &done[dev] : nullptr;
-  if (slot && slot->load(std::memory_order_acquire) == gen) return cudaSuccess;
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e == cudaSuccess && slot) slot->store(gen, std::memory_order_release);
-  return e;
-}
+// One record per kernel (a static of each kernel's launch function).
+struct SmemLimitRecord {
+  std::atomic<uint32_t> done[64];     // generation in which each device was set
+  template <typename K>
+  cudaError_t ensure(K kern, int bytes) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint32_t gen = g_setup_generation.load(std::memory_order_acquire);
+    std::atomic<uint32_t> *slot = dev >= 0 && dev < 64 ? &done[dev] : nullptr;
+    if (slot && slot->load(std::memory_order_acquire) == gen) return cudaSuccess;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && slot) slot->store(gen, std::memory_order_release);
+    return e;
+  }
+};
 
 // Launch with programmatic stream serialization: the kernel may begin (its
 // prologue) while the previous launch on the stream finishes; every kernel of

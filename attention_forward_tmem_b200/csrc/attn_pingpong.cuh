@@ -556,7 +556,8 @@ template <typename T, int DQK, int DROPE, int DV, bool kFuse>
 cudaError_t launch_attn_pp(const AttnParams &p, int grid, cudaStream_t stream) {
   using Cfg = PPCfg<T, DQK, DROPE, DV, kFuse>;
   auto kern = attn_fwd_pp_kernel<T, DQK, DROPE, DV, kFuse>;
-  cudaError_t e = ensure_smem_limit(kern, Cfg::kSmemBytes);
+  static SmemLimitRecord limit;       // this kernel's
+  cudaError_t e = limit.ensure(kern, Cfg::kSmemBytes);
   if (e != cudaSuccess) return e;
   return launch_pdl(kern, dim3(grid), dim3(kPPThreads), Cfg::kSmemBytes, stream, p);
 }
