@@ -69,11 +69,18 @@ KERNEL_SOURCES = ["attention_forward_tmem_b200/csrc/attn_pingpong.cuh",
 # ----------------------------------------------------------------- helpers
 
 def measured_peaks():
+    """Peak denominators: the generated MEASURED_PEAKS.json when present
+    (its bf16 sustained figure under whichever key holds it), else the
+    fallback figures of this GPU pool."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         with open(p) as f:
             d = json.load(f)
-        return d, "measured"
+        out = dict(d)
+        if "bf16_tflops_sustained" not in out:
+            cand = [v for k, v in d.items() if "sustained" in k and "bf16" in k and isinstance(v, (int, float))]
+            out["bf16_tflops_sustained"] = cand[0] if cand else out["bf16_tflops"]
+        return out, "measured"
     return FALLBACK_PEAKS, "fallback"
 
 
@@ -633,14 +640,20 @@ def measure(wl, timer, args):
 
 
 def roofline_of(wl, ms, peaks, peak_kind):
-    # the attention kernel's own rate: per launch, or (rolling cache) per step
-    # of fused attention + cache-write kernels and their merge passes
+    """The attention kernel's own rate (per launch, or for the rolling cache per
+    step of fused attention + cache-write kernels and their merge passes)
+    against the dense bf16 peak.  The timed region is a loop of at least a
+    second, which runs under the 1 kW power cap, so the denominator is the
+    sustained GEMM figure; the burst one is given beside it."""
     achieved = wl.flops / (ms / 1e3) / 1e12
-    return {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
-            "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+    sustained, burst = peaks["bf16_tflops_sustained"], peaks["bf16_tflops"]
+    return {"bound": "tensor", "achieved": achieved, "peak": sustained,
+            "unit": "TFLOP/s", "frac": achieved / sustained,
+            "frac_of_burst_peak": achieved / burst, "burst_peak": burst,
             "traffic": profiled_traffic(wl.name),
-            "peak_source": f"{peak_kind} bf16 burst (MEASURED_PEAKS.json)"
-            if peak_kind == "measured" else "fallback 1.59 PFLOP/s",
+            "peak_source": (f"{peak_kind} bf16 sustained (MEASURED_PEAKS.json; seconds-long loop under "
+                            "the power cap, as this timed region is)")
+            if peak_kind == "measured" else "fallback 1.4 PFLOP/s sustained (1.59 burst)",
             "kernel": "wf::attn_fwd_pp_kernel" if wl.w.dtype == torch.bfloat16 else "wf::attn_fwd_kernel",
             "algorithmic_flops_per_launch": wl.flops}
 
@@ -717,7 +730,7 @@ def keep_mask_throughput(device, timer, peaks):
     api.device_status()
     tf = flops / (ms / 1e3) / 1e12
     return {"value": tf, "unit": "TFLOP/s", "ms_per_step": ms, "timed_blocks": blocks,
-            "frac_of_peak": tf / peaks["bf16_tflops"], "clocks": clocks,
+            "frac_of_peak": tf / peaks["bf16_tflops_sustained"], "clocks": clocks,
             "config": "B 4, 32/8 heads, L 4096, D 128, bf16, keep-mask [1,1,4096,4096] p_keep 0.8 "
                       "(all pairs computed)"}
 
@@ -823,7 +836,8 @@ def main():
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "bf16", "data": "synthetic (seeded N(0,1), see workloads.py)",
                 "config": cfg,
-                "pct_of_peak": {"measured_bf16": 100 * achieved / peaks["bf16_tflops"],
+                "pct_of_peak": {"bf16_sustained": 100 * achieved / peaks["bf16_tflops_sustained"],
+                                "bf16_burst": 100 * achieved / peaks["bf16_tflops"],
                                 "datasheet_bf16_2250": 100 * achieved / DATASHEET_BF16_TFLOPS},
                 "roofline": roofline, "cpu_baseline": cpu,
                 "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
