@@ -155,12 +155,14 @@ struct ProducerLog {
 // pipe (exp2_poly2) instead of the MUFU unit, in tiles without masked scores.
 // At head size 128 the MUFU rate alone (16 per clock per SM) makes one
 // tile's softmax as long as the other tile's two MMAs.
-template <int kEmuPer16>
+// kExplicit: the instance that reads explicit masks (p.mask_kind keep or
+// add); without it only no mask and the causal mask are handled.
+template <int kEmuPer16, bool kExplicit>
 __device__ __forceinline__ float softmax_row(const AttnParams &p, const TileInfo &ti, int32_t row,
                                              int32_t k0, const uint32_t (&sr)[128],
                                              float (&x)[128], float &m, float &l) {
   const bool causal = p.mask_kind == kMaskCausal;
-  const bool explicit_mask = p.mask_kind == kMaskKeep || p.mask_kind == kMaskAdd;
+  const bool explicit_mask = kExplicit && (p.mask_kind == kMaskKeep || p.mask_kind == kMaskAdd);
   const bool row_valid = row < ti.lq;
   int32_t lim = ti.lk - 1 - k0;                      // last visible column of this row
   if (causal) lim = min(lim, row + ti.off - k0);
@@ -182,7 +184,7 @@ __device__ __forceinline__ float softmax_row(const AttnParams &p, const TileInfo
 #pragma unroll
     for (int c = 0; c < 128; ++c)
       x[c] = (c <= lim) ? __uint_as_float(sr[c]) * p.scale_log2 : -INFINITY;
-  } else {
+  } else if constexpr (kExplicit) {
     const int64_t mrow = (int64_t)ti.b * p.m_sb + (int64_t)ti.h * p.m_sh + (int64_t)row * p.m_si;
     // A full tile of a mask whose keys are contiguous and 16-byte aligned is
     // read with 16-byte loads: a thread's 128 entries in a few vector loads

@@ -3,7 +3,7 @@
 #include "attn_pingpong.cuh"
 
 namespace wf {
-template cudaError_t launch_attn_pp<__nv_bfloat16, 96, 0, 64, false>(const AttnParams &, int, cudaStream_t);
-template cudaError_t launch_attn_pp<__nv_bfloat16, 96, 0, 96, false>(const AttnParams &, int, cudaStream_t);
-template cudaError_t launch_attn_pp<__nv_bfloat16, 96, 0, 128, false>(const AttnParams &, int, cudaStream_t);
+template cudaError_t launch_attn_pp<__nv_bfloat16, 96, 0, 64, kKindPlain>(const AttnParams &, int, cudaStream_t);
+template cudaError_t launch_attn_pp<__nv_bfloat16, 96, 0, 96, kKindPlain>(const AttnParams &, int, cudaStream_t);
+template cudaError_t launch_attn_pp<__nv_bfloat16, 96, 0, 128, kKindPlain>(const AttnParams &, int, cudaStream_t);
 }  // namespace wf

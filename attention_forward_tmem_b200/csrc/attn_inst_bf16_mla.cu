@@ -3,5 +3,5 @@
 #include "attn_pingpong.cuh"
 
 namespace wf {
-template cudaError_t launch_attn_pp<__nv_bfloat16, 128, 64, 128, false>(const AttnParams &, int, cudaStream_t);
+template cudaError_t launch_attn_pp<__nv_bfloat16, 128, 64, 128, kKindPlain>(const AttnParams &, int, cudaStream_t);
 }  // namespace wf

@@ -134,9 +134,15 @@ struct AttnKernel {
   int32_t unit_rows;     // query rows per work unit of this kernel
 };
 
-// Kernel for (ElemType, dqk, drope, dv), optionally the instance that also
-// writes a BlockKVCache chunk; launch == nullptr if none.
-AttnKernel find_attn_kernel(int dtype, int dqk, int drope, int dv, bool fused = false);
+// Instances of the 16-bit kernel: no mask or the in-kernel causal mask; the
+// same plus the write of a BlockKVCache chunk; explicit masks (boolean keep
+// or additive) read from memory.  Each instance carries only its own code:
+// with the explicit-mask paths compiled into the causal instance, ~20% of its
+// executed instructions were predicated-off mask address arithmetic.
+enum KernelKind : int32_t { kKindPlain = 0, kKindFuse = 1, kKindMask = 2 };
+
+// Kernel for (ElemType, dqk, drope, dv, kind); launch == nullptr if none.
+AttnKernel find_attn_kernel(int dtype, int dqk, int drope, int dv, int kind = kKindPlain);
 
 // V [rows, heads, batch] x d (element strides) -> V^T [batch][heads][d][ld] (fp32).
 cudaError_t launch_transpose_v(const float *v, int64_t s_row, int64_t s_head, int64_t s_batch,

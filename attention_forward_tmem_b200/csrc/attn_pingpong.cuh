@@ -38,12 +38,14 @@ constexpr uint32_t kPPOtherRegs = 120;       // warpgroup 2: producer, MMA, 2 id
 // launch: 384 threads x 168 registers = 64512 >= 2*128*200 + 128*96 = 63488
 static_assert(2 * 128 * kPPSoftmaxRegs + 128 * kPPOtherRegs <= kPPThreads * 168, "register split");
 
-// kFuse: the kernel instance that also writes a BlockKVCache chunk (key rows
-// [fuse_lo, fuse_hi) read from the chunk and stored into the cache); the
-// plain instance carries none of that code.
-template <typename T, int DQK, int DROPE, int DV, bool kFuse_ = false>
+// kKind (KernelKind): kKindFuse is the instance that also writes a
+// BlockKVCache chunk (key rows [fuse_lo, fuse_hi) read from the chunk and
+// stored into the cache), kKindMask the one that reads explicit masks; the
+// plain instance (no mask or causal) carries neither's code.
+template <typename T, int DQK, int DROPE, int DV, int kKind = kKindPlain>
 struct PPCfg {
-  static constexpr bool kFuse = kFuse_;
+  static constexpr bool kFuse = kKind == kKindFuse;
+  static constexpr bool kMask = kKind == kKindMask;
   static constexpr int kAtomE = 64;                       // bf16 elements per 128-byte row
   static constexpr int kKStep = 16;
   static constexpr int kQAtoms = (DQK + kAtomE - 1) / kAtomE;
@@ -423,7 +425,7 @@ __device__ void pp_mma(const AttnParams &p, uint8_t *smem, PPCtrl *ctl, uint32_t
 }
 
 // ------------------------------------------------------------------- softmax
-template <typename T, int DV, int kEmuPer16>
+template <typename T, int DV, int kEmuPer16, bool kExplicit>
 __device__ void pp_softmax(const AttnParams &p, PPCtrl *ctl, uint32_t tmem, int s) {
   const int32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int32_t r = threadIdx.x & 127;                  // row within the tile = TMEM lane
@@ -454,7 +456,7 @@ __device__ void pp_softmax(const AttnParams &p, PPCtrl *ctl, uint32_t tmem, int 
       uint32_t sr[128];
       tmem_ld_x128(s_addr, sr);
       float x[128];
-      const float alpha = softmax_row<kEmuPer16>(p, ti, row, (ti.kt0 + j) * kBlockN, sr, x, m, l);
+      const float alpha = softmax_row<kEmuPer16, kExplicit>(p, ti, row, (ti.kt0 + j) * kBlockN, sr, x, m, l);
       tmem_store_p<T>(s_addr, x);
       // S_s(j) done implies PV_s(j-1) done: O_s may be rescaled right away.
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) tmem_scale_row<DV>(o_addr, alpha);
@@ -477,9 +479,9 @@ __device__ void pp_softmax(const AttnParams &p, PPCtrl *ctl, uint32_t tmem, int 
 }
 
 // --------------------------------------------------------------------- kernel
-template <typename T, int DQK, int DROPE, int DV, bool kFuse>
+template <typename T, int DQK, int DROPE, int DV, int kKind>
 __global__ void __launch_bounds__(kPPThreads, 1) attn_fwd_pp_kernel(const __grid_constant__ AttnParams p) {
-  using Cfg = PPCfg<T, DQK, DROPE, DV, kFuse>;
+  using Cfg = PPCfg<T, DQK, DROPE, DV, kKind>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
@@ -522,7 +524,7 @@ __global__ void __launch_bounds__(kPPThreads, 1) attn_fwd_pp_kernel(const __grid
   ProducerLog plog;
   if (warp < 8) {
     regs_increase<kPPSoftmaxRegs>();
-    pp_softmax<T, DV, Cfg::kEmuPer16>(p, ctl, tmem, warp >> 2);
+    pp_softmax<T, DV, Cfg::kEmuPer16, Cfg::kMask>(p, ctl, tmem, warp >> 2);
   } else {
     regs_decrease<kPPOtherRegs>();
     if (warp == 8) pp_producer<Cfg>(p, smem, ctl, plog, elect_one());
@@ -552,10 +554,10 @@ __global__ void __launch_bounds__(kPPThreads, 1) attn_fwd_pp_kernel(const __grid
   }
 }
 
-template <typename T, int DQK, int DROPE, int DV, bool kFuse>
+template <typename T, int DQK, int DROPE, int DV, int kKind>
 cudaError_t launch_attn_pp(const AttnParams &p, int grid, cudaStream_t stream) {
-  using Cfg = PPCfg<T, DQK, DROPE, DV, kFuse>;
-  auto kern = attn_fwd_pp_kernel<T, DQK, DROPE, DV, kFuse>;
+  using Cfg = PPCfg<T, DQK, DROPE, DV, kKind>;
+  auto kern = attn_fwd_pp_kernel<T, DQK, DROPE, DV, kKind>;
   static SmemLimitRecord limit;       // this kernel's
   cudaError_t e = limit.ensure(kern, Cfg::kSmemBytes);
   if (e != cudaSuccess) return e;

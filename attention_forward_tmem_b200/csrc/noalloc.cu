@@ -120,7 +120,7 @@ extern "C" wf_status_t wf_attn_fwd_varlen_noalloc(
     if (!(drope == 64 && dqk == 128 && dv == 128))
       return fail(WF_ERR_UNSUPPORTED, "rope part needs Dqk = Dv = 128 and a 64-wide rope");
   }
-  const AttnKernel kern = find_attn_kernel(1, (int)dqk, (int)drope, (int)dv);
+  const AttnKernel kern = find_attn_kernel(kElemBF16, (int)dqk, (int)drope, (int)dv, kKindPlain);
   if (!kern.launch)
     return fail(WF_ERR_UNSUPPORTED, "head sizes Dqk=%lld Dv=%lld are not implemented",
                 (long long)dqk, (long long)dv);

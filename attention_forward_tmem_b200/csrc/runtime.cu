@@ -485,7 +485,8 @@ static wf_status_t attn_fwd_impl(const wf_tensor_t *q, const wf_tensor_t *qRope,
   // supported head sizes
   if (d.drope && !(d.drope == 64 && d.dqk == 128 && d.dv == 128 && dt != WF_F32))
     return fail(WF_ERR_UNSUPPORTED, "rope part needs 16-bit inputs, Dqk = Dv = 128 and a 64-wide rope");
-  AttnKernel kern = find_attn_kernel(elem_type(dt), (int)d.dqk, (int)d.drope, (int)d.dv);
+  AttnKernel kern = find_attn_kernel(elem_type(dt), (int)d.dqk, (int)d.drope, (int)d.dv,
+                                     explicit_mask ? kKindMask : kKindPlain);
   if (!kern.launch)
     return fail(WF_ERR_UNSUPPORTED, "head sizes Dqk=%lld Dv=%lld (rope %lld) are not implemented",
                 (long long)d.dqk, (long long)d.dv, (long long)d.drope);
@@ -505,7 +506,7 @@ static wf_status_t attn_fwd_impl(const wf_tensor_t *q, const wf_tensor_t *qRope,
     if (fuse->k_chunk->shape[3] != d.dqk || fuse->v_chunk->shape[3] != d.dv)
       return fail(WF_ERR_INVALID_ARG, "chunk head sizes differ from k / v");
     // the kernel instance that also writes the chunk, where one is built
-    const AttnKernel fk = find_attn_kernel(elem_type(dt), (int)d.dqk, 0, (int)d.dv, true);
+    const AttnKernel fk = find_attn_kernel(elem_type(dt), (int)d.dqk, 0, (int)d.dv, kKindFuse);
     if (!fk.launch) {
       *fuse->declined = true;
       return WF_OK;
