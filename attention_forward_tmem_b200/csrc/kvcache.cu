@@ -12,9 +12,11 @@
 // chunk_size and the window holds at least one chunk; update takes exactly
 // chunk_size positions; chunk c lives in slot c while c < sink/chunk and in
 // sink/chunk + (c - sink/chunk) mod (window/chunk) afterwards.
+#include <algorithm>
 #include <cstdint>
 #include <cstring>
 #include <new>
+#include <type_traits>
 
 #include "attn_params.h"
 #include "runtime.h"
@@ -65,66 +67,139 @@ View logical(const wf_tensor_t *t, int32_t seq_dim) {
   return v;
 }
 
-// Copy `rows` = B*H*C rows of `row_bytes` each: source row (b, h, t) ->
-// destination row (b, h, dst_t0 + t).  `unit` bytes per thread step (16, 8, 4,
-// 2 or 1, chosen on the host so every access is aligned to it).
-template <typename U>
-__global__ void copy_rows_kernel(const uint8_t *__restrict__ src, int64_t s_b, int64_t s_h,
-                                 int64_t s_t, uint8_t *__restrict__ dst, int64_t d_b, int64_t d_h,
-                                 int64_t d_t, int64_t dst_t0, int64_t H, int64_t C, int64_t n_rows,
-                                 int64_t units_per_row) {
+// Copy jobs: `rows` = B*H*C rows of `upr` units each, source row (b, h, t) ->
+// destination row (b, h, dst_t0 + t); strides in bytes.  One launch runs up
+// to two jobs (the chunk's K and V), one per grid row.
+struct CopyJob {
+  const uint8_t *src;
+  uint8_t *dst;
+  int64_t s_b, s_h, s_t, d_b, d_h, d_t, dst_t0, upr, total;
+};
+struct CopyJobs {
+  CopyJob job[2];
+  int64_t H, C;
+};
+
+// `unit` bytes (U) per element, chosen on the host so every access is aligned
+// to it; each thread keeps four elements' loads in flight before it stores
+// them.  kNarrow: element counts and row counts fit 32 bits, so the index
+// arithmetic is 32-bit.
+template <typename U, bool kNarrow>
+__global__ void __launch_bounds__(256) copy_rows_kernel(const __grid_constant__ CopyJobs cj) {
   pdl_wait();
   pdl_trigger();
-  const int64_t total = n_rows * units_per_row;
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t row = i / units_per_row, u = i - row * units_per_row;
-    const int64_t t = row % C, h = (row / C) % H, b = row / (C * H);
-    const U *s = reinterpret_cast<const U *>(src + b * s_b + h * s_h + t * s_t) + u;
-    U *d = reinterpret_cast<U *>(dst + b * d_b + h * d_h + (dst_t0 + t) * d_t) + u;
-    *d = *s;
+  const CopyJob &j = cj.job[blockIdx.y];
+  using I = typename std::conditional<kNarrow, uint32_t, int64_t>::type;
+  const I upr = static_cast<I>(j.upr), C = static_cast<I>(cj.C), H = static_cast<I>(cj.H);
+  const I total = static_cast<I>(j.total);
+  const I stride = static_cast<I>(gridDim.x) * blockDim.x;
+  for (I base = static_cast<I>(blockIdx.x) * blockDim.x + threadIdx.x; base < total; base += 4 * stride) {
+    U v[4];
+    U *d[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const I i = base + k * stride;
+      d[k] = nullptr;
+      if (i < total) {
+        const I row = i / upr, u = i - row * upr;
+        const I t = row % C, bh = row / C;
+        const I h = bh % H, b = bh / H;
+        v[k] = *(reinterpret_cast<const U *>(j.src + (int64_t)b * j.s_b + (int64_t)h * j.s_h + (int64_t)t * j.s_t) + u);
+        d[k] = reinterpret_cast<U *>(j.dst + (int64_t)b * j.d_b + (int64_t)h * j.d_h +
+                                     (j.dst_t0 + (int64_t)t) * j.d_t) + u;
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (d[k]) *d[k] = v[k];
   }
 }
 
+// One copy: C positions of every (b, h) row from src (starting at src_t0) to
+// dst (starting at dst_t0); views are logical [B, H, L, D].
+struct CopyReq {
+  const void *src_base;
+  View s;
+  int64_t src_t0;
+  void *dst_base;
+  View d;
+  int64_t dst_t0;
+};
+
+// Largest power of two (at most 16) that divides x.
 int64_t gcd_pow2_unit(int64_t x) {
   for (int64_t u = 16; u > 1; u >>= 1)
     if (x % u == 0) return u;
   return 1;
 }
 
-// Copy C positions of every (b, h) row from src (starting at src_t0) to dst
-// (starting at dst_t0).  Views are logical [B, H, L, D].
-wf_status_t copy_positions(const void *src_base, const View &s, int64_t src_t0, void *dst_base,
-                           const View &d, int64_t dst_t0, int64_t C, size_t es,
-                           cudaStream_t stream) {
-  const int64_t rows = s.B * s.H * C;
-  if (rows == 0 || s.D == 0) return WF_OK;
-  const int64_t row_bytes = s.D * (int64_t)es;
-  const uint8_t *src = static_cast<const uint8_t *>(src_base) + src_t0 * s.sl * (int64_t)es;
-  uint8_t *dst = static_cast<uint8_t *>(dst_base);
+static int64_t unit_of(const CopyReq &r, size_t es) {
+  const int64_t row_bytes = r.s.D * (int64_t)es;
   int64_t unit = gcd_pow2_unit(row_bytes);
+  const uint8_t *src = static_cast<const uint8_t *>(r.src_base) + r.src_t0 * r.s.sl * (int64_t)es;
   const int64_t vals[] = {(int64_t)reinterpret_cast<uintptr_t>(src),
-                          (int64_t)reinterpret_cast<uintptr_t>(dst), s.sb * (int64_t)es,
-                          s.sh * (int64_t)es, s.sl * (int64_t)es, d.sb * (int64_t)es,
-                          d.sh * (int64_t)es, d.sl * (int64_t)es};
+                          (int64_t)reinterpret_cast<uintptr_t>(r.dst_base), r.s.sb * (int64_t)es,
+                          r.s.sh * (int64_t)es, r.s.sl * (int64_t)es, r.d.sb * (int64_t)es,
+                          r.d.sh * (int64_t)es, r.d.sl * (int64_t)es};
   for (int64_t x : vals)
     while (unit > 1 && x % unit != 0) unit >>= 1;
-  const int64_t upr = row_bytes / unit;
-  const int64_t total = rows * upr;
+  return unit;
+}
+
+static CopyJob job_of(const CopyReq &r, int64_t C, size_t es, int64_t unit) {
+  CopyJob j;
+  j.src = static_cast<const uint8_t *>(r.src_base) + r.src_t0 * r.s.sl * (int64_t)es;
+  j.dst = static_cast<uint8_t *>(r.dst_base);
+  j.s_b = r.s.sb * es; j.s_h = r.s.sh * es; j.s_t = r.s.sl * es;
+  j.d_b = r.d.sb * es; j.d_h = r.d.sh * es; j.d_t = r.d.sl * es;
+  j.dst_t0 = r.dst_t0;
+  j.upr = r.s.D * (int64_t)es / unit;
+  j.total = r.s.B * r.s.H * C * j.upr;
+  return j;
+}
+
+template <typename U>
+static cudaError_t launch_copy(const CopyJobs &cj, int n_jobs, int64_t max_total, cudaStream_t stream) {
   const int threads = 256;
-  int64_t blocks = (total + threads - 1) / threads;
-  if (blocks > 148 * 16) blocks = 148 * 16;
-  const int64_t sb = s.sb * es, sh = s.sh * es, st = s.sl * es;
-  const int64_t db = d.sb * es, dh = d.sh * es, dt = d.sl * es;
-  cudaError_t e;
-  switch (unit) {
-    case 16: e = launch_pdl(copy_rows_kernel<uint4>, dim3((unsigned)blocks), dim3(threads), 0, stream, src, sb, sh, st, dst, db, dh, dt, dst_t0, s.H, C, rows, upr); break;
-    case 8: e = launch_pdl(copy_rows_kernel<uint2>, dim3((unsigned)blocks), dim3(threads), 0, stream, src, sb, sh, st, dst, db, dh, dt, dst_t0, s.H, C, rows, upr); break;
-    case 4: e = launch_pdl(copy_rows_kernel<uint32_t>, dim3((unsigned)blocks), dim3(threads), 0, stream, src, sb, sh, st, dst, db, dh, dt, dst_t0, s.H, C, rows, upr); break;
-    case 2: e = launch_pdl(copy_rows_kernel<uint16_t>, dim3((unsigned)blocks), dim3(threads), 0, stream, src, sb, sh, st, dst, db, dh, dt, dst_t0, s.H, C, rows, upr); break;
-    default: e = launch_pdl(copy_rows_kernel<uint8_t>, dim3((unsigned)blocks), dim3(threads), 0, stream, src, sb, sh, st, dst, db, dh, dt, dst_t0, s.H, C, rows, upr); break;
+  int64_t blocks = (max_total + 4 * threads - 1) / (4 * threads);
+  if (blocks > 148 * 8) blocks = 148 * 8;
+  const dim3 grid((unsigned)blocks, (unsigned)n_jobs);
+  const bool narrow = max_total < (int64_t(1) << 31) && cj.C < (int64_t(1) << 31) && cj.H < (int64_t(1) << 31);
+  if (narrow) return launch_pdl(copy_rows_kernel<U, true>, grid, dim3(threads), 0, stream, cj);
+  return launch_pdl(copy_rows_kernel<U, false>, grid, dim3(threads), 0, stream, cj);
+}
+
+// Copy one or two requests (K and V of a chunk) of C positions each; both in
+// one launch when their element sizes agree, else one launch each.
+wf_status_t copy_positions(const CopyReq *reqs, int n, int64_t C, size_t es, cudaStream_t stream) {
+  CopyReq live[2];
+  int m = 0;
+  for (int i = 0; i < n; ++i)
+    if (reqs[i].s.B * reqs[i].s.H * C > 0 && reqs[i].s.D > 0) live[m++] = reqs[i];
+  if (m == 0) return WF_OK;
+  int64_t units[2] = {unit_of(live[0], es), m > 1 ? unit_of(live[1], es) : 0};
+  const bool together = m == 2 && units[0] == units[1];
+  for (int first = 0; first < m; first += together ? 2 : 1) {
+    const int cnt = together ? 2 : 1;
+    const int64_t unit = units[first];
+    CopyJobs cj{};
+    cj.H = live[first].s.H;
+    cj.C = C;
+    int64_t max_total = 0;
+    for (int k = 0; k < cnt; ++k) {
+      cj.job[k] = job_of(live[first + k], C, es, unit);
+      max_total = std::max(max_total, cj.job[k].total);
+    }
+    cudaError_t e;
+    switch (unit) {
+      case 16: e = launch_copy<uint4>(cj, cnt, max_total, stream); break;
+      case 8: e = launch_copy<uint2>(cj, cnt, max_total, stream); break;
+      case 4: e = launch_copy<uint32_t>(cj, cnt, max_total, stream); break;
+      case 2: e = launch_copy<uint16_t>(cj, cnt, max_total, stream); break;
+      default: e = launch_copy<uint8_t>(cj, cnt, max_total, stream); break;
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "cache copy launch");
   }
-  if (e != cudaSuccess) return cuda_fail(e, "cache copy launch");
   return WF_OK;
 }
 
@@ -226,12 +301,11 @@ wf_status_t wf_kvcache_update(wf_kvcache_t *c, const wf_tensor_t *k, const wf_te
   const int64_t t0 = slot_of(c, c->current) * c->chunk;
   const size_t es = dtype_size(c->k.dtype);
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  if ((st = copy_positions(k->data, logical(k, c->seq_dim), 0, c->k.data, logical(&c->k, c->seq_dim),
-                           t0, c->chunk, es, cs)) != WF_OK)
-    return st;
-  if ((st = copy_positions(v->data, logical(v, c->seq_dim), 0, c->v.data, logical(&c->v, c->seq_dim),
-                           t0, c->chunk, es, cs)) != WF_OK)
-    return st;
+  {
+    const CopyReq reqs[2] = {{k->data, logical(k, c->seq_dim), 0, c->k.data, logical(&c->k, c->seq_dim), t0},
+                             {v->data, logical(v, c->seq_dim), 0, c->v.data, logical(&c->v, c->seq_dim), t0}};
+    if ((st = copy_positions(reqs, 2, c->chunk, es, cs)) != WF_OK) return st;
+  }
   c->phase = kUpdated;
   return WF_OK;
 }
@@ -271,12 +345,9 @@ wf_status_t wf_kvcache_update_attend(wf_kvcache_t *c, const wf_tensor_t *k, cons
   if (declined) {                               // not fusable: the copies, then the attention
     const size_t es = dtype_size(c->k.dtype);
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    if ((st = copy_positions(k->data, logical(k, c->seq_dim), 0, c->k.data, logical(&c->k, c->seq_dim),
-                             lo, c->chunk, es, cs)) != WF_OK)
-      return st;
-    if ((st = copy_positions(v->data, logical(v, c->seq_dim), 0, c->v.data, logical(&c->v, c->seq_dim),
-                             lo, c->chunk, es, cs)) != WF_OK)
-      return st;
+    const CopyReq reqs[2] = {{k->data, logical(k, c->seq_dim), 0, c->k.data, logical(&c->k, c->seq_dim), lo},
+                             {v->data, logical(v, c->seq_dim), 0, c->v.data, logical(&c->v, c->seq_dim), lo}};
+    if ((st = copy_positions(reqs, 2, c->chunk, es, cs)) != WF_OK) return st;
     if ((st = wf_attn_fwd(q, nullptr, &kv, nullptr, &vv, nullptr, nullptr, nullptr, headNum, kv_heads,
                           qkScale, WF_MASK_NONE, out, stream)) != WF_OK)
       return st;
@@ -350,11 +421,10 @@ wf_status_t wf_kvcache_gather_logical(wf_kvcache_t *c, wf_tensor_t *k_out, wf_te
   int64_t pos = 0;
   auto emit = [&](int64_t idx) -> wf_status_t {
     const int64_t src_t0 = slot_of(c, idx) * c->chunk;
-    wf_status_t s2 = copy_positions(c->k.data, logical(&c->k, c->seq_dim), src_t0, k_out->data,
-                                    logical(k_out, c->seq_dim), pos * c->chunk, c->chunk, es, cs);
-    if (s2 == WF_OK)
-      s2 = copy_positions(c->v.data, logical(&c->v, c->seq_dim), src_t0, v_out->data,
-                          logical(v_out, c->seq_dim), pos * c->chunk, c->chunk, es, cs);
+    const CopyReq reqs[2] = {
+        {c->k.data, logical(&c->k, c->seq_dim), src_t0, k_out->data, logical(k_out, c->seq_dim), pos * c->chunk},
+        {c->v.data, logical(&c->v, c->seq_dim), src_t0, v_out->data, logical(v_out, c->seq_dim), pos * c->chunk}};
+    wf_status_t s2 = copy_positions(reqs, 2, c->chunk, es, cs);
     ++pos;
     return s2;
   };
