@@ -133,6 +133,21 @@ __device__ __forceinline__ bool pp_next_item(const AttnParams &p, PPCtrl *ctl, u
   return true;
 }
 
+// Dense launches with p.unit_major: the counter's k-th claim takes the k-th
+// item in unit-rank-major order (the longest unit of every (batch, kv head)
+// block, then the next, ...), mapped here to its index in the block-major
+// enumeration that tile_info decodes.  Claim k = ((j * blocks + blk) * G +
+// head in group) * n_split + split; item = ((blk * units + j) * G + head) *
+// n_split + split.
+__device__ __forceinline__ int32_t unit_major_item(const AttnParams &p, int32_t k) {
+  const int32_t S = p.n_split > 1 ? p.n_split : 1;
+  const int32_t G = p.group, blocks = p.batch * p.hkv;
+  const int32_t u = k / S, sp = k - u * S;
+  const int32_t q = u / G, hh = u - q * G;
+  const int32_t j = q / blocks, blk = q - j * blocks;
+  return ((blk * p.units_per_bh + j) * G + hh) * S + sp;
+}
+
 // ------------------------------------------------------------------ producer
 // Runs on all lanes of warp 8; `leader` (one lane) issues the copies.
 template <typename Cfg>
@@ -210,6 +225,7 @@ __device__ void pp_producer(const AttnParams &p, uint8_t *smem, PPCtrl *ctl, Pro
     int32_t t = 0;
     if (leader) t = atomicAdd(p.counters, 1);
     t = __shfl_sync(0xffffffffu, t, leader_lane);
+    if (p.unit_major && t < n_units) t = unit_major_item(p, t);
     TileInfo t0, t1;
     if (t < n_units) {
       t0 = tile_info(p, t, 0);

@@ -74,7 +74,8 @@ DeviceState *current_device_state(wf_status_t *st) {
   DeviceState ds;
   if ((e = cudaDeviceGetAttribute(&ds.sm_count, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
       (e = cudaDeviceGetAttribute(&ds.cc_major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
-      (e = cudaDeviceGetAttribute(&ds.cc_minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess) {
+      (e = cudaDeviceGetAttribute(&ds.cc_minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess ||
+      (e = cudaDeviceGetAttribute(&ds.l2_bytes, cudaDevAttrL2CacheSize, dev)) != cudaSuccess) {
     *st = cuda_fail(e, "cudaDeviceGetAttribute");
     return nullptr;
   }
@@ -673,6 +674,21 @@ static wf_status_t attn_fwd_impl(const wf_tensor_t *q, const wf_tensor_t *qRope,
       return fail(WF_ERR_UNSUPPORTED, "too many work items (%lld)", (long long)(units * n_split));
     p.units_per_bh = (int32_t)per_bh;
     p.n_units_dense = (int32_t)units;
+    // Causal units differ in length.  Block by block (locality first), with
+    // fewer items in a (batch, kv head) block than SMs, several blocks run at
+    // once and the last blocks' longest units start near the end of the
+    // launch, leaving SMs idle while they finish (c2: 64 items a block on 148
+    // SMs; ncu: SM active 93% of the elapsed cycles).  There, when the K and
+    // V of all blocks fit in ~60% of L2 together, items go by unit length
+    // over the whole launch (c2 +2.4%).  With more items a block than SMs the
+    // last block fills the machine, longest first, by itself, and the block
+    // order keeps fewer K / V tensors in use (unit rank order there: -2.3%
+    // at 64 / 8 heads, L 16 384).
+    const double kv_bytes = (double)d.batch * kvHeadNum * n_keys * (d.dqk + d.drope + d.dv) * dtype_size(dt);
+    p.unit_major = p.mask_kind == kMaskCausal && per_bh > 1 && per_bh * (headNum / kvHeadNum) < ds->sm_count &&
+                           kv_bytes <= 0.6 * ds->l2_bytes
+                       ? 1
+                       : 0;
     if (units * n_split < grid) grid = (int)(units * n_split);
   } else {
     const int64_t B = d.batch;

@@ -22,6 +22,7 @@ size_t dtype_size(int32_t dtype);
 // Per-device state: SM count, status word address.
 struct DeviceState {
   int sm_count = 0;
+  int l2_bytes = 0;
   int cc_major = 0, cc_minor = 0;
   int32_t *status = nullptr;     // address of the device status word
 };
