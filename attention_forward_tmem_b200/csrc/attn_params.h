@@ -62,8 +62,8 @@ struct alignas(64) AttnParams {
   int32_t kv_padded;                             // packed q, K/V [batch, max_seq, heads, D]
   int32_t unit_rows;                             // query rows per work unit (128 or 256)
   int32_t n_units_dense, units_per_bh;           // dense: total units, units per (b, h)
-  int32_t unit_major;                            // dense: items claimed by unit rank across all
-                                                 // (batch, kv head) blocks (see unit_major_item)
+  int32_t unit_major;                            // dense: the last unit_major (batch, kv head)
+                                                 // blocks claimed by unit rank (unit_major_item)
   const int32_t *ws;                             // varlen schedule (device)
   int32_t *counters;                             // two-tile kernel: [next item, CTAs done],
                                                  // zero before a launch, zero after it

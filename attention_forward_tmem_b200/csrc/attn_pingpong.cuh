@@ -133,18 +133,22 @@ __device__ __forceinline__ bool pp_next_item(const AttnParams &p, PPCtrl *ctl, u
   return true;
 }
 
-// Dense launches with p.unit_major: the counter's k-th claim takes the k-th
-// item in unit-rank-major order (the longest unit of every (batch, kv head)
-// block, then the next, ...), mapped here to its index in the block-major
-// enumeration that tile_info decodes.  Claim k = ((j * blocks + blk) * G +
-// head in group) * n_split + split; item = ((blk * units + j) * G + head) *
-// n_split + split.
+// Dense launches with p.unit_major = W > 0: claims go through the (batch, kv
+// head) blocks in order, except the last W blocks, whose items are claimed in
+// unit-rank order (the longest unit of each of the W blocks, then the next,
+// ...), so that the launch ends on short units.  Mapped here to the index of
+// the item in the block-major enumeration that tile_info decodes: within the
+// last W blocks claim k = ((j * W + b) * G + head in group) * n_split +
+// split; item = ((blk * units + j) * G + head) * n_split + split, blk =
+// blocks - W + b.
 __device__ __forceinline__ int32_t unit_major_item(const AttnParams &p, int32_t k) {
   const int32_t S = p.n_split > 1 ? p.n_split : 1;
-  const int32_t G = p.group, blocks = p.batch * p.hkv;
-  const int32_t u = k / S, sp = k - u * S;
+  const int32_t G = p.group, blocks = p.batch * p.hkv, W = p.unit_major;
+  const int32_t k0 = (blocks - W) * p.units_per_bh * G * S;
+  if (k < k0) return k;
+  const int32_t u = (k - k0) / S, sp = (k - k0) - u * S;
   const int32_t q = u / G, hh = u - q * G;
-  const int32_t j = q / blocks, blk = q - j * blocks;
+  const int32_t j = q / W, blk = blocks - W + (q - j * W);
   return ((blk * p.units_per_bh + j) * G + hh) * S + sp;
 }
 

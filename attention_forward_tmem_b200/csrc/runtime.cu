@@ -678,17 +678,18 @@ static wf_status_t attn_fwd_impl(const wf_tensor_t *q, const wf_tensor_t *qRope,
     // fewer items in a (batch, kv head) block than SMs, several blocks run at
     // once and the last blocks' longest units start near the end of the
     // launch, leaving SMs idle while they finish (c2: 64 items a block on 148
-    // SMs; ncu: SM active 93% of the elapsed cycles).  There, when the K and
-    // V of all blocks fit in ~60% of L2 together, items go by unit length
-    // over the whole launch (c2 +2.4%).  With more items a block than SMs the
-    // last block fills the machine, longest first, by itself, and the block
-    // order keeps fewer K / V tensors in use (unit rank order there: -2.3%
-    // at 64 / 8 heads, L 16 384).
-    const double kv_bytes = (double)d.batch * kvHeadNum * n_keys * (d.dqk + d.drope + d.dv) * dtype_size(dt);
-    p.unit_major = p.mask_kind == kMaskCausal && per_bh > 1 && per_bh * (headNum / kvHeadNum) < ds->sm_count &&
-                           kv_bytes <= 0.6 * ds->l2_bytes
-                       ? 1
-                       : 0;
+    // SMs; ncu: SM active 93% of the elapsed cycles).  There the last blocks,
+    // about two waves of items, are claimed by unit rank instead, so the
+    // launch ends on short units (SM active 98%).  Only those blocks: in unit
+    // rank order over all 32 blocks of c2 the K / V of every block stayed in
+    // use, were read ~3 times, and the extra DRAM power cost the gain back
+    // under the power cap.  With more items a block than SMs the last block
+    // fills the machine, longest first, by itself.
+    const int64_t items_per_block = per_bh * (headNum / kvHeadNum);
+    const int64_t blocks = d.batch * kvHeadNum;
+    p.unit_major = 0;
+    if (p.mask_kind == kMaskCausal && per_bh > 1 && blocks > 1 && items_per_block < ds->sm_count)
+      p.unit_major = (int32_t)std::min<int64_t>(blocks, (2 * ds->sm_count + items_per_block - 1) / items_per_block);
     if (units * n_split < grid) grid = (int)(units * n_split);
   } else {
     const int64_t B = d.batch;
