@@ -50,6 +50,10 @@ struct alignas(64) AttnParams {
   // each kv head store them into tm_k / tm_v.  fuse_hi == 0: no fusion.
   CUtensorMap tm_kc, tm_vc;
   int32_t fuse_lo, fuse_hi;
+  // Dense output through TMA stores (tma_out != 0): map of out (Dv, Lq, Hq,
+  // B) with 64 x 32 boxes; the kernel uses it where it has the staging area.
+  CUtensorMap tm_o;
+  int32_t tma_out;
   void *out;
   int64_t o_sb, o_sh, o_si;                      // element strides of out (batch, head, row)
   const void *mask;

@@ -64,7 +64,14 @@ struct PPCfg {
   static constexpr int kVStages = kEqFit >= 3 ? 3 : (kEqFit == 2 ? 2 : 1);
   static constexpr int kKOff = kQBytes;
   static constexpr int kVOff = kKOff + kKStages * kKBytes;
-  static constexpr int kCtrlOff = kVOff + kVStages * kVBytes;
+  // Output staging (p.tma_out): a 4 KB area per softmax warp, its 32 rows x
+  // 64 columns of O in bf16 / f16 (128-byte swizzle), stored to global
+  // memory by the tensor-memory accelerator one half row at a time; head
+  // size 128 only, where it fits beside the rings.
+  static constexpr int kStageOff = kVOff + kVStages * kVBytes;
+  static constexpr bool kTmaEpi =
+      DV == 128 && kStageOff + 8 * 4096 + 1024 + 1024 <= 227 * 1024;
+  static constexpr int kCtrlOff = kStageOff + (kTmaEpi ? 8 * 4096 : 0);
   static constexpr int kSmemUsed = kCtrlOff + 1024 + 1024;
   static constexpr int kSmemBytes = kSmemUsed > 120 * 1024 ? kSmemUsed : 120 * 1024;
   static constexpr int kSKStepsQK = DQK / kKStep;
@@ -487,8 +494,43 @@ __device__ void pp_mma(const AttnParams &p, uint8_t *smem, PPCtrl *ctl, uint32_t
 }
 
 // ------------------------------------------------------------------- softmax
-template <typename T, int DV, int kEmuPer16, bool kExplicit>
-__device__ void pp_softmax(const AttnParams &p, PPCtrl *ctl, uint32_t tmem, int s) {
+// Epilogue through shared memory (p.tma_out, dense, no split): the warp's 32
+// rows of O / l, each row in two 64-column halves, written as 16-bit pairs
+// into its 4 KB staging area in the 128-byte swizzle of the output map and
+// stored by one lane with a TMA tensor store (rows past Lq are clipped by the
+// map).  With one thread per row, direct stores make every warp store
+// instruction touch 32 rows (~1 000 store transactions per tile and item on
+// the softmax warps' path); a half-row box is 4 KB in one bulk copy.
+template <typename T, int DV>
+__device__ __forceinline__ void store_rows_tma(const AttnParams &p, const TileInfo &ti, uint8_t *stage,
+                                               const float (&o)[DV], float inv, int32_t row0) {
+  static_assert(DV == 128, "two 64-column halves");
+  const int lane = threadIdx.x & 31;
+  const uint32_t base = smem_u32(stage) + lane * 128u;
+#pragma unroll
+  for (int hf = 0; hf < 2; ++hf) {
+    if (lane == 0) bulk_wait_read();            // the area is free again (previous store read it)
+    __syncwarp();
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const float *v = o + hf * 64 + c * 8;
+      const uint32_t w0 = Elem16<T>::pack2(v[0] * inv, v[1] * inv), w1 = Elem16<T>::pack2(v[2] * inv, v[3] * inv);
+      const uint32_t w2 = Elem16<T>::pack2(v[4] * inv, v[5] * inv), w3 = Elem16<T>::pack2(v[6] * inv, v[7] * inv);
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(base + ((c ^ (lane & 7)) << 4)), "r"(w0),
+                   "r"(w1), "r"(w2), "r"(w3)
+                   : "memory");
+    }
+    fence_proxy_async();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_4d(&p.tm_o, stage, hf * 64, row0, ti.h, ti.b);
+      bulk_commit_group();
+    }
+  }
+}
+
+template <typename T, int DV, int kEmuPer16, bool kExplicit, bool kTmaEpi>
+__device__ void pp_softmax(const AttnParams &p, PPCtrl *ctl, uint32_t tmem, int s, uint8_t *stage) {
   const int32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int32_t r = threadIdx.x & 127;                  // row within the tile = TMEM lane
   const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
@@ -536,8 +578,20 @@ __device__ void pp_softmax(const AttnParams &p, PPCtrl *ctl, uint32_t tmem, int 
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(&ctl->o_empty[s]);
+    if constexpr (kTmaEpi) {
+      if (p.tma_out) {
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        store_rows_tma<T, DV>(p, ti, stage, o, inv, ti.q0 + (warp & 3) * 32);
+        if (row_valid && p.lse)
+          p.lse[(int64_t)ti.b * p.l_sb + (int64_t)ti.h * p.l_sh + (int64_t)row * p.l_si] =
+              l > 0.f ? (m + __log2f(l)) * kLn2 : -INFINITY;
+        continue;
+      }
+    }
     if (row_valid) store_result<T, DV>(p, ti, row, o, m, l);
   }
+  if constexpr (kTmaEpi)
+    if (lane == 0) bulk_wait_all();               // the output stores are done before the CTA ends
 }
 
 // --------------------------------------------------------------------- kernel
@@ -586,7 +640,8 @@ __global__ void __launch_bounds__(kPPThreads, 1) attn_fwd_pp_kernel(const __grid
   ProducerLog plog;
   if (warp < 8) {
     regs_increase<kPPSoftmaxRegs>();
-    pp_softmax<T, DV, Cfg::kEmuPer16, Cfg::kMask>(p, ctl, tmem, warp >> 2);
+    pp_softmax<T, DV, Cfg::kEmuPer16, Cfg::kMask, Cfg::kTmaEpi>(p, ctl, tmem, warp >> 2,
+                                                                smem + Cfg::kStageOff + warp * 4096);
   } else {
     regs_decrease<kPPOtherRegs>();
     if (warp == 8) pp_producer<Cfg>(p, smem, ctl, plog, elect_one());

@@ -169,14 +169,14 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // swizzle, zero fill outside the tensor.  Strides in elements.
 wf_status_t make_map(CUtensorMap *map, const void *base, int32_t dtype, int64_t d,
                             int64_t rows, int64_t heads, int64_t batch, int64_t s_row,
-                            int64_t s_head, int64_t s_batch, const char *name) {
+                            int64_t s_head, int64_t s_batch, const char *name, int32_t box_rows) {
   auto fn = encode_fn();
   if (!fn) return fail(WF_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   const size_t es = dtype_size(dtype);
   const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)heads, (cuuint64_t)batch};
   const cuuint64_t strides[3] = {(cuuint64_t)(s_row * es), (cuuint64_t)(s_head * es),
                                  (cuuint64_t)(s_batch * es)};
-  const cuuint32_t box[4] = {(cuuint32_t)(128 / es), (cuuint32_t)kBlockM, 1, 1};
+  const cuuint32_t box[4] = {(cuuint32_t)(128 / es), (cuuint32_t)box_rows, 1, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   const CUtensorMapDataType dt = dtype == WF_F32    ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
                                  : dtype == WF_F16  ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
@@ -569,6 +569,17 @@ static wf_status_t attn_fwd_impl(const wf_tensor_t *q, const wf_tensor_t *qRope,
     p.o_sb = out->stride[0];
     p.o_sh = out->stride[1];
     p.o_si = out->stride[2];
+    // Output rows through shared memory and TMA stores (two-tile kernel,
+    // head size 128, no split; see pp_softmax): where the map's rules hold
+    // (16-byte aligned base, strides multiples of 16 bytes), 32-row boxes.
+    const int64_t es = (int64_t)dtype_size(dt);
+    const auto al16 = [&](int64_t v) { return (v * es) % 16 == 0; };
+    if (dt != WF_F32 && d.dv == 128 && d.lq > 0 && (reinterpret_cast<uintptr_t>(out->data) & 15) == 0 &&
+        al16(p.o_si) && al16(p.o_sh) && al16(p.o_sb) && p.o_si > 0 && p.o_sh > 0 && p.o_sb > 0 &&
+        make_map(&p.tm_o, out->data, dt, d.dv, d.lq, headNum, d.batch, p.o_si, p.o_sh, p.o_sb, "out", 32) == WF_OK)
+      p.tma_out = 1;
+    else
+      clear_error();
   } else {
     p.o_sb = 0;
     p.o_sh = out->stride[1];
@@ -610,6 +621,7 @@ static wf_status_t attn_fwd_impl(const wf_tensor_t *q, const wf_tensor_t *qRope,
     n_split = (int32_t)std::max<int64_t>(1, std::min(by_grid, by_len));
   }
   p.n_split = n_split;
+  if (n_split > 1) p.tma_out = 0;           // partial rows in fp32 go to the workspace
 
   // Per-stream workspace: [schedule tables (varlen)] [V^T (fp32)] [split
   // partials: out fp32, lse fp32], 256-byte aligned parts.

@@ -60,6 +60,6 @@ void forget_noalloc_addresses();
 // 128-byte swizzle, zero fill outside the tensor; strides in elements.
 wf_status_t make_map(CUtensorMap *map, const void *base, int32_t dtype, int64_t d, int64_t rows,
                      int64_t heads, int64_t batch, int64_t s_row, int64_t s_head, int64_t s_batch,
-                     const char *name);
+                     const char *name, int32_t box_rows = 128);
 
 }  // namespace wf
