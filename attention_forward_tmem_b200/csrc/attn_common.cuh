@@ -404,12 +404,19 @@ __device__ __forceinline__ void store_zero_row(const AttnParams &p, const TileIn
 // Load DV fp32 columns of this thread's TMEM lane starting at `taddr`.
 template <int DV>
 __device__ __forceinline__ void tmem_load_row(uint32_t taddr, float (&o)[DV]) {
+  if constexpr (DV == 128) {      // one load and one wait for the whole row
+    uint32_t oc[128];
+    tmem_ld_x128(taddr, oc);
 #pragma unroll
-  for (int c0 = 0; c0 < DV; c0 += 32) {
-    uint32_t oc[32];
-    tmem_ld_x32(taddr + c0, oc);
+    for (int c = 0; c < 128; ++c) o[c] = __uint_as_float(oc[c]);
+  } else {
 #pragma unroll
-    for (int c = 0; c < 32; ++c) o[c0 + c] = __uint_as_float(oc[c]);
+    for (int c0 = 0; c0 < DV; c0 += 32) {
+      uint32_t oc[32];
+      tmem_ld_x32(taddr + c0, oc);
+#pragma unroll
+      for (int c = 0; c < 32; ++c) o[c0 + c] = __uint_as_float(oc[c]);
+    }
   }
 }
 
