@@ -54,6 +54,10 @@ struct alignas(64) AttnParams {
   // B) with 64 x 32 boxes; the kernel uses it where it has the staging area.
   CUtensorMap tm_o;
   int32_t tma_out;
+  // Split-KV partial rows through TMA stores (tma_part != 0, dense): map of
+  // part_o (Dv, part_rows, n_split) in fp32 with 32 x 32 boxes.
+  CUtensorMap tm_po;
+  int32_t tma_part;
   void *out;
   int64_t o_sb, o_sh, o_si;                      // element strides of out (batch, head, row)
   const void *mask;

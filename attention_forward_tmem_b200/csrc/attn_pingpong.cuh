@@ -529,6 +529,37 @@ __device__ __forceinline__ void store_rows_tma(const AttnParams &p, const TileIn
   }
 }
 
+// The same for split-KV partial rows (p.tma_part, dense): fp32 O / l of the
+// split in four 32-column quarters (128 bytes of each row), stored into
+// part_o at row part_rows index r0 (the warp's first row) and split `sp`.
+// Only for warps whose 32 rows all lie below Lq: the partial rows of one
+// (batch, head) are followed by the next head's.
+template <int DV>
+__device__ __forceinline__ void store_part_rows_tma(const AttnParams &p, uint8_t *stage, const float (&o)[DV],
+                                                    float inv, int64_t r0, int32_t sp) {
+  static_assert(DV == 128, "four 32-column quarters");
+  const int lane = threadIdx.x & 31;
+  const uint32_t base = smem_u32(stage) + lane * 128u;
+#pragma unroll
+  for (int qt = 0; qt < 4; ++qt) {
+    if (lane == 0) bulk_wait_read();
+    __syncwarp();
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const float *v = o + qt * 32 + c * 4;
+      asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(base + ((c ^ (lane & 7)) << 4)),
+                   "f"(v[0] * inv), "f"(v[1] * inv), "f"(v[2] * inv), "f"(v[3] * inv)
+                   : "memory");
+    }
+    fence_proxy_async();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_4d(&p.tm_po, stage, qt * 32, static_cast<int32_t>(r0), sp, 0);
+      bulk_commit_group();
+    }
+  }
+}
+
 template <typename T, int DV, int kEmuPer16, bool kExplicit, bool kTmaEpi>
 __device__ void pp_softmax(const AttnParams &p, PPCtrl *ctl, uint32_t tmem, int s, uint8_t *stage) {
   const int32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -585,6 +616,14 @@ __device__ void pp_softmax(const AttnParams &p, PPCtrl *ctl, uint32_t tmem, int 
         if (row_valid && p.lse)
           p.lse[(int64_t)ti.b * p.l_sb + (int64_t)ti.h * p.l_sh + (int64_t)row * p.l_si] =
               l > 0.f ? (m + __log2f(l)) * kLn2 : -INFINITY;
+        continue;
+      }
+      const int32_t row0 = ti.q0 + (warp & 3) * 32;
+      if (p.tma_part && p.n_split > 1 && !p.varlen && row0 + 32 <= ti.lq) {
+        const int64_t r0 = ((int64_t)ti.b * p.hq + ti.h) * p.lq + row0;
+        store_part_rows_tma<DV>(p, stage, o, l > 0.f ? 1.f / l : 0.f, r0, ti.sp);
+        p.part_lse[(int64_t)ti.sp * p.part_rows + r0 + (r & 31)] =
+            l > 0.f ? (m + __log2f(l)) * kLn2 : -INFINITY;
         continue;
       }
     }

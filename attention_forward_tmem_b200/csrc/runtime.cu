@@ -655,6 +655,13 @@ static wf_status_t attn_fwd_impl(const wf_tensor_t *q, const wf_tensor_t *qRope,
     p.part_o = reinterpret_cast<float *>(base);
     p.part_lse = reinterpret_cast<float *>(base + part_o_bytes);
     p.part_rows = part_rows;
+    // the two-tile kernel's staged stores of partial rows (dense, head size 128)
+    if (!d.varlen && dt != WF_F32 && d.dv == 128 &&
+        make_map(&p.tm_po, p.part_o, WF_F32, d.dv, part_rows, n_split, 1, d.dv, part_rows * d.dv,
+                 (int64_t)n_split * part_rows * d.dv, "split partials", 32) == WF_OK)
+      p.tma_part = 1;
+    else
+      clear_error();
   }
   if (dt == WF_F32) {
     float *vt = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(ws) + sched_bytes);
