@@ -157,10 +157,29 @@ struct ProducerLog {
 // tile's softmax as long as the other tile's two MMAs.
 // kExplicit: the instance that reads explicit masks (p.mask_kind keep or
 // add); without it only no mask and the causal mask are handled.
-template <int kEmuPer16, bool kExplicit>
+// kPSplit > 0: `mid(alpha)` is called once p_0 .. p_{kPSplit-1} are final,
+// before the remaining columns are exponentiated (the caller hands that part
+// of P to the PV product early).
+template <int C0, int C1, int kEmuPer16>
+__device__ __forceinline__ void exp_cols(float (&x)[128], float (&sq)[8], float sc, float neg_m) {
+#pragma unroll
+  for (int c = C0; c < C1; c += 2) {
+    fma2_bc(x[c], x[c + 1], x[c], x[c + 1], sc, neg_m);
+    if ((c & 15) < kEmuPer16) {
+      exp2_poly2(x[c], x[c + 1]);
+    } else {
+      x[c] = ex2_approx(x[c]);
+      x[c + 1] = ex2_approx(x[c + 1]);
+    }
+    const int q = (c >> 1) & 3;
+    add2(sq[2 * q], sq[2 * q + 1], x[c], x[c + 1]);
+  }
+}
+
+template <int kEmuPer16, bool kExplicit, int kPSplit = 0, typename Mid>
 __device__ __forceinline__ float softmax_row(const AttnParams &p, const TileInfo &ti, int32_t row,
                                              int32_t k0, const uint32_t (&sr)[128],
-                                             float (&x)[128], float &m, float &l) {
+                                             float (&x)[128], float &m, float &l, Mid &&mid) {
   const bool causal = p.mask_kind == kMaskCausal;
   const bool explicit_mask = kExplicit && (p.mask_kind == kMaskKeep || p.mask_kind == kMaskAdd);
   const bool row_valid = row < ti.lq;
@@ -287,27 +306,13 @@ __device__ __forceinline__ float softmax_row(const AttnParams &p, const TileInfo
   const float sc = prescaled ? 1.f : p.scale_log2;
   float sq[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   if (kEmuPer16 > 0 && !prescaled && !need_mask) {
-#pragma unroll
-    for (int c = 0; c < 128; c += 2) {
-      fma2_bc(x[c], x[c + 1], x[c], x[c + 1], sc, neg_m);
-      if ((c & 15) < kEmuPer16) {
-        exp2_poly2(x[c], x[c + 1]);
-      } else {
-        x[c] = ex2_approx(x[c]);
-        x[c + 1] = ex2_approx(x[c + 1]);
-      }
-      const int q = (c >> 1) & 3;
-      add2(sq[2 * q], sq[2 * q + 1], x[c], x[c + 1]);
-    }
+    exp_cols<0, kPSplit, kEmuPer16>(x, sq, sc, neg_m);
+    if constexpr (kPSplit > 0) mid(alpha);
+    exp_cols<kPSplit, 128, kEmuPer16>(x, sq, sc, neg_m);
   } else {
-#pragma unroll
-    for (int c = 0; c < 128; c += 2) {
-      fma2_bc(x[c], x[c + 1], x[c], x[c + 1], sc, neg_m);
-      x[c] = ex2_approx(x[c]);
-      x[c + 1] = ex2_approx(x[c + 1]);
-      const int q = (c >> 1) & 3;
-      add2(sq[2 * q], sq[2 * q + 1], x[c], x[c + 1]);
-    }
+    exp_cols<0, kPSplit, 0>(x, sq, sc, neg_m);
+    if constexpr (kPSplit > 0) mid(alpha);
+    exp_cols<kPSplit, 128, 0>(x, sq, sc, neg_m);
   }
   const float sum = ((sq[0] + sq[1]) + (sq[2] + sq[3])) + ((sq[4] + sq[5]) + (sq[6] + sq[7]));
   l = l * alpha + sum;
@@ -450,6 +455,26 @@ __device__ __forceinline__ void tmem_store_p(uint32_t taddr, const float (&x)[12
 #pragma unroll
     for (int c = 0; c < 64; ++c) pk[c] = __float_as_uint(x[64 + c]);
     tmem_st_x64(taddr + 64, pk);
+  }
+}
+
+// P values [C0, C1) of the row (16-bit pairs) into TMEM columns C0/2 ..
+// C1/2 of the score slot at `taddr`, where the PV product reads keys C0 .. C1;
+// stored as 32-, 16- and 8-column pieces.
+template <typename T, int C0, int C1>
+__device__ __forceinline__ void tmem_store_p_part(uint32_t taddr, const float (&x)[128]) {
+  static_assert(sizeof(T) == 2 && C0 % 16 == 0 && C1 % 16 == 0 && C0 <= C1 && C1 <= 128, "P part");
+  constexpr int N = (C1 - C0) / 2;
+  if constexpr (N > 0) {
+    uint32_t pk[N];
+#pragma unroll
+    for (int c = 0; c < N; ++c) pk[c] = Elem16<T>::pack2(x[C0 + 2 * c], x[C0 + 2 * c + 1]);
+    constexpr int n64 = N & 64, n32 = N & 32, n16 = N & 16;
+    const uint32_t a = taddr + C0 / 2;
+    if constexpr (n64 != 0) tmem_st_x64(a, *reinterpret_cast<const uint32_t(*)[64]>(pk));
+    if constexpr (n32 != 0) tmem_st_x32(a + n64, *reinterpret_cast<const uint32_t(*)[32]>(pk + n64));
+    if constexpr (n16 != 0) tmem_st_x16(a + n64 + n32, pk + n64 + n32);
+    if constexpr ((N & 8) != 0) tmem_st_x8(a + n64 + n32 + n16, pk + n64 + n32 + n16);
   }
 }
 

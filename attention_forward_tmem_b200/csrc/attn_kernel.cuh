@@ -264,7 +264,8 @@ __device__ void softmax_role(const AttnParams &p, AttnCtrl *ctl, uint32_t tmem) 
       uint32_t sr[128];
       tmem_ld_x128(tmem + lane_base + sb * 128, sr);
       float x[128];
-      const float alpha = softmax_row<0, true>(p, ti, row, (ti.kt0 + j) * kBlockN, sr, x, m, l);
+      const float alpha = softmax_row<0, true>(p, ti, row, (ti.kt0 + j) * kBlockN, sr, x, m, l,
+                                                 [](float) {});
       tmem_store_p<T>(tmem + lane_base + sb * 128, x);
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
         // O holds the sum up to tile j-1 once PV[gg-1] is done.

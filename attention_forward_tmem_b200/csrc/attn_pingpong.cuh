@@ -85,13 +85,23 @@ struct PPCfg {
   // suspend instead of spinning, a share of 4/16 cost ~4% at head size 128
   // and more with the 192-wide MLA product, so the MUFU unit does all of them.
   static constexpr int kEmuPer16 = 0;
+  // Keys of P handed to the PV product ahead of the rest: the softmax warps
+  // store p_0 .. p_{kPSplit-1} and signal p_part before exponentiating the
+  // remaining columns, so the MMA warp issues those k-steps of PV while they
+  // are computed and only the rest of PV and the next S product stay on the
+  // path from the last P value to the next scores.  Measured on B200 (short
+  // runs): 80 of 128 keys gave c2 +2.4%, the L 16 384 GQA case +3.7% and the
+  // rolling cache loop +0.6% (64, 96 and 112 were within 0.5% of it); with a
+  // rope part (MLA) every split cost ~1%, so that instance hands P over whole.
+  static constexpr int kPSplit = kRAtoms > 0 ? 0 : 80;
   static_assert(kKStages >= 1 && kVStages >= 1 && kSmemUsed <= 227 * 1024, "smem");
   static_assert(DQK % kKStep == 0 && DV % 32 == 0 && kNPV <= 128, "head dims");
+  static_assert(kPSplit % kKStep == 0 && kPSplit >= 0 && kPSplit < kBlockN, "P split");
 };
 
 struct PPCtrl {
   uint64_t q_full, q_empty, drain;
-  uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
+  uint64_t s_full[2], p_part[2], p_full[2], o_full[2], o_empty[2];
   uint64_t k_full[3], k_empty[3], v_full[3], v_empty[3];
   uint64_t sched_full[2], sched_empty[2];
   volatile int32_t sched_item[2];
@@ -297,11 +307,11 @@ struct IssueS {
   }
 };
 // O (+)= P V: P read from TMEM (8 columns per k-step), V MN-major (16 rows of
-// 128 bytes per k-step).
-template <typename Cfg, int KS>
+// 128 bytes per k-step); k-steps K0..KS.
+template <typename Cfg, int K0, int KS>
 struct IssuePV {
   static __device__ __forceinline__ void run(uint32_t d, uint32_t p_tmem, Desc v, uint32_t acc0) {
-    if constexpr (KS > 0) IssuePV<Cfg, KS - 1>::run(d, p_tmem, v, acc0);
+    if constexpr (KS > K0) IssuePV<Cfg, K0, KS - 1>::run(d, p_tmem, v, acc0);
     mma_f16_ts_at<KS * 8, ((KS * Cfg::kKStep * 128) >> 4)>(d, p_tmem, v, Cfg::kIdescPV,
                                                          KS > 0 ? 1u : acc0);
   }
@@ -312,10 +322,12 @@ __device__ __forceinline__ void pp_issue_s(uint32_t tmem, Desc q, Desc k, int s)
   IssueS<Cfg, Cfg::kSKStepsQK + Cfg::kSKStepsR - 1>::run(tmem + (s ? 128u : 0u), q, k);
 }
 
-template <typename Cfg>
+// k-steps [K0, K1) of PV (keys 16 K0 .. 16 K1 of the tile).
+template <typename Cfg, int K0, int K1>
 __device__ __forceinline__ void pp_issue_pv(uint32_t tmem, Desc v, int s, bool accumulate) {
-  IssuePV<Cfg, Cfg::kPVKSteps - 1>::run(tmem + (s ? 384u : 256u), tmem + (s ? 128u : 0u), v,
-                                        accumulate ? 1u : 0u);
+  if constexpr (K1 > K0)
+    IssuePV<Cfg, K0, K1 - 1>::run(tmem + (s ? 384u : 256u), tmem + (s ? 128u : 0u), v,
+                                  accumulate ? 1u : 0u);
 }
 
 template <typename Cfg>
@@ -370,10 +382,16 @@ __device__ void pp_mma(const AttnParams &p, uint8_t *smem, PPCtrl *ctl, uint32_t
   };
   // PV of tile slot s for KV tile (unit-local) jj; returns false on abort.
   auto do_pv = [&](int s, int32_t jj, int32_t n_s, uint32_t gg) -> bool {
+    constexpr int kSplitSteps = Cfg::kPSplit / Cfg::kKStep;
     if (jj == 0 && !bwait_w(&ctl->o_empty[s], (co[s] + 1) & 1, &ctl->abort, p)) return false;
+    if constexpr (kSplitSteps > 0) {
+      if (!bwait_w(&ctl->p_part[s], cp[s] & 1, &ctl->abort, p)) return false;
+      tc_fence_after();
+      if (leader) pp_issue_pv<Cfg, 0, kSplitSteps>(tmem, vbase(gg), s, jj > 0);
+    }
     if (!bwait_w(&ctl->p_full[s], cp[s] & 1, &ctl->abort, p)) return false;
     tc_fence_after();
-    if (leader) pp_issue_pv<Cfg>(tmem, vbase(gg), s, jj > 0);
+    if (leader) pp_issue_pv<Cfg, kSplitSteps, Cfg::kPVKSteps>(tmem, vbase(gg), s, jj > 0);
     ++cp[s];
     if (jj == n_s - 1 && leader) tc_commit(&ctl->o_full[s]);
     return true;
@@ -560,7 +578,7 @@ __device__ __forceinline__ void store_part_rows_tma(const AttnParams &p, uint8_t
   }
 }
 
-template <typename T, int DV, int kEmuPer16, bool kExplicit, bool kTmaEpi>
+template <typename T, int DV, int kEmuPer16, bool kExplicit, bool kTmaEpi, int kPSplit>
 __device__ void pp_softmax(const AttnParams &p, PPCtrl *ctl, uint32_t tmem, int s, uint8_t *stage) {
   const int32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int32_t r = threadIdx.x & 127;                  // row within the tile = TMEM lane
@@ -591,10 +609,20 @@ __device__ void pp_softmax(const AttnParams &p, PPCtrl *ctl, uint32_t tmem, int 
       uint32_t sr[128];
       tmem_ld_x128(s_addr, sr);
       float x[128];
-      const float alpha = softmax_row<kEmuPer16, kExplicit>(p, ti, row, (ti.kt0 + j) * kBlockN, sr, x, m, l);
-      tmem_store_p<T>(s_addr, x);
-      // S_s(j) done implies PV_s(j-1) done: O_s may be rescaled right away.
-      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) tmem_scale_row<DV>(o_addr, alpha);
+      // S_s(j) done implies PV_s(j-1) done: O_s may be rescaled right away,
+      // before any part of P_s(j) is handed to PV_s(j).
+      auto first_part = [&](float a) {
+        tmem_store_p_part<T, 0, kPSplit>(s_addr, x);
+        if (j > 0 && __any_sync(0xffffffffu, a != 1.f)) tmem_scale_row<DV>(o_addr, a);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->p_part[s]);
+      };
+      const float alpha = softmax_row<kEmuPer16, kExplicit, kPSplit>(p, ti, row, (ti.kt0 + j) * kBlockN,
+                                                                     sr, x, m, l, first_part);
+      tmem_store_p_part<T, kPSplit, 128>(s_addr, x);
+      if (kPSplit == 0 && j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) tmem_scale_row<DV>(o_addr, alpha);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -649,6 +677,7 @@ __global__ void __launch_bounds__(kPPThreads, 1) attn_fwd_pp_kernel(const __grid
     mbar_init(&ctl->drain, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&ctl->s_full[i], 1);
+      mbar_init(&ctl->p_part[i], 4);
       mbar_init(&ctl->p_full[i], 4);
       mbar_init(&ctl->o_full[i], 1);
       mbar_init(&ctl->o_empty[i], 4);
@@ -679,7 +708,7 @@ __global__ void __launch_bounds__(kPPThreads, 1) attn_fwd_pp_kernel(const __grid
   ProducerLog plog;
   if (warp < 8) {
     regs_increase<kPPSoftmaxRegs>();
-    pp_softmax<T, DV, Cfg::kEmuPer16, Cfg::kMask, Cfg::kTmaEpi>(p, ctl, tmem, warp >> 2,
+    pp_softmax<T, DV, Cfg::kEmuPer16, Cfg::kMask, Cfg::kTmaEpi, Cfg::kPSplit>(p, ctl, tmem, warp >> 2,
                                                                 smem + Cfg::kStageOff + warp * 4096);
   } else {
     regs_decrease<kPPOtherRegs>();
