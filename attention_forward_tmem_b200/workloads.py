@@ -106,6 +106,29 @@ def dense_inputs(batch, head_num, kv_head_num, lq, lk, dqk, dv, dtype=torch.bflo
     return q, k, v
 
 
+def growing_score_inputs(batch, head_num, kv_head_num, lq, lk, dqk, dv, dtype=torch.bfloat16,
+                         seed=SEED, growth=0.02, q_bias=4.0, noise=0.5, drope=0):
+    """Dense q, k, v whose scores grow along the key index, so that an online
+    softmax raises its running row maximum on every key tile: every query
+    carries q_bias * u and key j carries growth * j * u, for one shared unit
+    vector u, over N(0, noise^2) entries; q_i . k_j is then ~q_bias * growth * j
+    plus noise (with the defaults and qk_scale 1, ~15 log2 units more per
+    128 keys).  drope > 0 appends N(0, noise^2) rope parts qRope [B,Hq,Lq,drope]
+    and kRope [B,Hkv,Lk,drope] to the returned tuple."""
+    g = _gen(seed)
+    u = torch.randn(dqk, generator=g, dtype=torch.float32)
+    u = u / u.norm()
+    q = _randn(g, (batch, head_num, lq, dqk), torch.float32, noise) + q_bias * u
+    j = torch.arange(lk, dtype=torch.float32).view(1, 1, lk, 1)
+    k = _randn(g, (batch, kv_head_num, lk, dqk), torch.float32, noise) + growth * j * u
+    v = _randn(g, (batch, kv_head_num, lk, dv), dtype)
+    if drope:
+        qr = _randn(g, (batch, head_num, lq, drope), dtype, noise)
+        kr = _randn(g, (batch, kv_head_num, lk, drope), dtype, noise)
+        return q.to(dtype), k.to(dtype), v, qr, kr
+    return q.to(dtype), k.to(dtype), v
+
+
 def seqlens(batch, lo, hi, seed=SEED):
     """Per-sequence lengths uniform in [lo, hi] (inclusive)."""
     g = _gen(seed)

@@ -69,6 +69,47 @@ def test_dense_bf16(cfg):
     compare(out, ref, torch.bfloat16, str(cfg))
 
 
+GROWING = [
+    # B, Hq, Hk, Lq, Lk, D, Dv, mask, num_splits
+    (1, 4, 2, 640, 640, 128, 128, "causal", None),
+    (1, 4, 2, 300, 700, 128, 128, "none", None),
+    (1, 2, 2, 256, 1024, 128, 128, "none", 3),       # split-KV partials and the merge
+    (1, 2, 1, 200, 333, 64, 64, "causal", None),
+    (1, 2, 2, 333, 200, 96, 128, "none", None),
+]
+
+
+@pytest.mark.parametrize("cfg", GROWING, ids=lambda c: "x".join(map(str, c)))
+def test_running_max_grows_every_tile(cfg):
+    """Scores that grow along the key index: the running row maximum rises by
+    more than the lazy-rescale threshold (2^8) on every 128-key tile, so O is
+    rescaled in tensor memory on every step, before that step's P (or the part
+    of it handed over first) reaches the PV product."""
+    B, Hq, Hk, Lq, Lk, D, Dv, mk, ns = cfg
+    q, k, v = W.growing_score_inputs(B, Hq, Hk, Lq, Lk, D, Dv)
+    mt = api.MaskType.CAUSAL if mk == "causal" else api.MaskType.NONE
+    out = api.attn_fwd(q.to(DEV), k.to(DEV), v.to(DEV), mask_type=mt, qk_scale=1.0, num_splits=ns)
+    api.device_status()
+    ref = oracle.sdpa(q, k, v, mask_kind=mk, qk_scale=1.0)
+    compare(out, ref, torch.bfloat16, str(cfg))
+
+
+def test_running_max_grows_every_tile_mla_packed():
+    """The same growth through the rope instance (packed, one sequence):
+    that instance hands P to the PV product whole."""
+    H, L = 4, 520
+    q, k, v, qr, kr = W.growing_score_inputs(1, H, H, L, L, 128, 128, drope=64)
+    pk = lambda t: t[0].transpose(0, 1).contiguous()  # noqa: E731  [1,H,L,D] -> [L,H,D]
+    lens = torch.tensor([L], dtype=torch.int32)
+    out = api.attn_fwd(pk(q).to(DEV), pk(k).to(DEV), pk(v).to(DEV), qrope=pk(qr).to(DEV),
+                       krope=pk(kr).to(DEV), q_seqlen=lens.to(DEV), kv_seqlen=lens.to(DEV),
+                       mask_type=api.MaskType.CAUSAL, qk_scale=1.0)
+    api.device_status()
+    ref = oracle.sdpa(pk(q), pk(k), pk(v), qrope=pk(qr), krope=pk(kr), q_seqlen=lens, kv_seqlen=lens,
+                      mask_kind="causal", qk_scale=1.0)
+    compare(out, ref, torch.bfloat16, "growing scores, MLA packed")
+
+
 DENSE_F32 = [
     (1, 4, 2, 300, 270, 128, 128, "causal"),     # one pipeline stage (large fp32 tiles)
     (2, 2, 2, 50, 77, 96, 96, "none"),
