@@ -94,6 +94,50 @@ def test_running_max_grows_every_tile(cfg):
     compare(out, ref, torch.bfloat16, str(cfg))
 
 
+@pytest.mark.parametrize("kind", ["keep", "add"])
+def test_running_max_grows_every_tile_masked(kind):
+    """Growing scores through the explicit-mask instance, whose softmax step
+    scales the scores (and adds the mask) before taking the row maximum."""
+    B, Hq, Hk, Lq, Lk = 1, 4, 2, 300, 640
+    q, k, v = W.growing_score_inputs(B, Hq, Hk, Lq, Lk, 128, 128)
+    g = torch.Generator().manual_seed(13)
+    if kind == "keep":
+        m = torch.rand(1, 1, Lq, Lk, generator=g) < 0.8
+    else:
+        m = torch.randn(1, 1, Lq, Lk, generator=g).to(torch.bfloat16)
+    out = api.attn_fwd(q.to(DEV), k.to(DEV), v.to(DEV), mask=m.to(DEV), qk_scale=1.0)
+    api.device_status()
+    ref = oracle.sdpa(q, k, v, mask=m.float() if kind == "add" else m, mask_kind=kind, qk_scale=1.0)
+    compare(out, ref, torch.bfloat16, f"growing scores, {kind} mask")
+
+
+@pytest.mark.parametrize("mk", ["causal", "none"])
+def test_running_max_grows_every_tile_negative_scale(mk):
+    """A negative qk_scale: the plain instance then scales the scores before
+    the row maximum (max and a negative factor do not commute).  q carries
+    -4u, so qk_scale * q.k still grows along the key index."""
+    q, k, v = W.growing_score_inputs(1, 4, 2, 400, 640, 128, 128, q_bias=-4.0)
+    mt = api.MaskType.CAUSAL if mk == "causal" else api.MaskType.NONE
+    out = api.attn_fwd(q.to(DEV), k.to(DEV), v.to(DEV), mask_type=mt, qk_scale=-1.0)
+    api.device_status()
+    ref = oracle.sdpa(q, k, v, mask_kind=mk, qk_scale=-1.0)
+    compare(out, ref, torch.bfloat16, f"growing scores, qk_scale -1, {mk}")
+
+
+def test_zero_scale_gives_the_mean_of_visible_values():
+    """qk_scale 0: every visible key has the same weight, so each output row is
+    the mean of the V rows its causal range covers (checked against the
+    oracle and against that mean directly)."""
+    q, k, v = W.dense_inputs(1, 2, 1, 300, 300, 128, 128, torch.bfloat16, 21)
+    out = api.attn_fwd(q.to(DEV), k.to(DEV), v.to(DEV), mask_type=api.MaskType.CAUSAL, qk_scale=0.0)
+    api.device_status()
+    ref = oracle.sdpa(q, k, v, mask_kind="causal", qk_scale=0.0)
+    compare(out, ref, torch.bfloat16, "qk_scale 0")
+    vf = v[0, 0].double().numpy()
+    mean = np.cumsum(vf, axis=0) / np.arange(1, 301)[:, None]
+    assert np.abs(ref[0, 0] - mean).max() < 1e-9 and np.abs(ref[0, 1] - mean).max() < 1e-9
+
+
 def test_running_max_grows_every_tile_mla_packed():
     """The same growth through the rope instance (packed, one sequence):
     that instance hands P to the PV product whole."""
