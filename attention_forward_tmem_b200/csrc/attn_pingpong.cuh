@@ -90,9 +90,10 @@ struct PPCfg {
   // remaining columns, so the MMA warp issues those k-steps of PV while they
   // are computed and only the rest of PV and the next S product stay on the
   // path from the last P value to the next scores.  Measured on B200 (short
-  // runs): 80 of 128 keys gave c2 +2.4%, the L 16 384 GQA case +3.7% and the
-  // rolling cache loop +0.6% (64, 96 and 112 were within 0.5% of it); with a
-  // rope part (MLA) every split cost ~1%, so that instance hands P over whole.
+  // runs): 80 of 128 keys gave +2.4% on the causal GQA prefill (B 4, 32/8
+  // heads, L 4096, D 128), +3.7% on the 64/8-head one at L 16 384 and +0.6% on
+  // the rolling cache loop (64, 96 and 112 keys were within 0.5% of 80); with
+  // a rope part (MLA) every split cost ~1%, so that instance hands P over whole.
   static constexpr int kPSplit = kRAtoms > 0 ? 0 : 80;
   static_assert(kKStages >= 1 && kVStages >= 1 && kSmemUsed <= 227 * 1024, "smem");
   static_assert(DQK % kKStep == 0 && DV % 32 == 0 && kNPV <= 128, "head dims");
@@ -402,7 +403,8 @@ __device__ void pp_mma(const AttnParams &p, uint8_t *smem, PPCtrl *ctl, uint32_t
   // right away and, once its Q and first K tile are in, its S_A(0) is issued
   // before B's last P is waited for, so tile A's softmax starts the next item
   // as soon as its epilogue is done instead of idling through B's extra step
-  // (clock64 trace, c2: ~6 400 cycles a boundary; c2 +1.6%).  `taken`: the
+  // (clock64 trace of the causal GQA prefill at B 4, 32/8 heads, L 4096:
+  // ~6 400 cycles a boundary; +1.6% there).  `taken`: the
   // next item is in t_next / tis_next; `early`: its Q and K0 were waited for
   // and its S_A(0) issued.  Not in the fused instance, whose stores follow the
   // item, nor with a rope part: that S product is 1.5 times longer, and ahead

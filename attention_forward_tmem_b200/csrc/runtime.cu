@@ -696,11 +696,12 @@ static wf_status_t attn_fwd_impl(const wf_tensor_t *q, const wf_tensor_t *qRope,
     // Causal units differ in length.  Block by block (locality first), with
     // fewer items in a (batch, kv head) block than SMs, several blocks run at
     // once and the last blocks' longest units start near the end of the
-    // launch, leaving SMs idle while they finish (c2: 64 items a block on 148
-    // SMs; ncu: SM active 93% of the elapsed cycles).  There the last blocks,
+    // launch, leaving SMs idle while they finish (causal GQA prefill at B 4,
+    // 32/8 heads, L 4096: 64 items a block on 148 SMs; ncu: SM active 93% of
+    // the elapsed cycles).  There the last blocks,
     // about two waves of items, are claimed by unit rank instead, so the
     // launch ends on short units (SM active 98%).  Only those blocks: in unit
-    // rank order over all 32 blocks of c2 the K / V of every block stayed in
+    // rank order over all 32 blocks of that workload the K / V of every block stayed in
     // use, were read ~3 times, and the extra DRAM power cost the gain back
     // under the power cap.  With more items a block than SMs the last block
     // fills the machine, longest first, by itself.
